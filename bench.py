@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Benchmark of the persistent warp-specialized BF16 GEMM (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload square8192|square4096|llm_up|llm_down|edge4099|edge8192x256|
+                                edge127x8191|recsys|square256|all]
+
+A step is one GEMM (one launch of the persistent kernel) over the workload's synthetic
+inputs, already resident in HBM.  Timing: W untimed warm-up steps, then K steps between
+CUDA events on the launching stream, bracketed by a barrier and a device synchronize; the
+time is the max over ranks.  Multi-GPU runs are independent replicas (the GEMM needs no
+exchange): value = total FLOPs of all ranks / max time.  `--impl reference` times the fp64
+CPU oracle (rank 0 only) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GEMM TFLOP/s (bf16 in, fp32 acc) and % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+SPEC_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+L2_BYTES = 126 * 2 ** 20
+
+# name -> (description, batch, M, N, K, out, alpha, beta, std_a, std_b, dist, config index)
+WORKLOADS = {
+    "square256": ("single GEMM M=N=K=256, U[-1,1], fp32 out", 1, 256, 256, 256, "f32", 1.0, 0.0,
+                  1.0, 1.0, "uniform", 0),
+    "square4096": ("square GEMM M=N=K=4096, N(0,1), bf16 out", 1, 4096, 4096, 4096, "bf16", 1.0, 0.0,
+                   1.0, 1.0, "normal", 1),
+    "square8192": ("square GEMM M=N=K=8192, N(0,1), bf16 out", 1, 8192, 8192, 8192, "bf16", 1.0, 0.0,
+                   1.0, 1.0, "normal", 1),
+    "llm_up": ("LLM MLP up-proj M=16384 N=28672 K=8192, act N(0,1), W N(0,0.02), bf16 out", 1, 16384,
+               28672, 8192, "bf16", 1.0, 0.0, 1.0, 0.02, "normal", 2),
+    "llm_down": ("LLM MLP down-proj M=16384 N=8192 K=28672, act N(0,1), W N(0,0.02), bf16 out", 1,
+                 16384, 8192, 28672, "bf16", 1.0, 0.0, 1.0, 0.02, "normal", 2),
+    "edge4099": ("edge GEMM M=N=K=4099 packed ld, alpha=0.5 beta=1, bf16 C in place", 1, 4099, 4099,
+                 4099, "bf16", 0.5, 1.0, 1.0, 1.0, "normal", 3),
+    "edge8192x256": ("edge GEMM M=8192 N=256 K=4096, alpha=0.5 beta=1, bf16 C in place", 1, 8192, 256,
+                     4096, "bf16", 0.5, 1.0, 1.0, 1.0, "normal", 3),
+    "edge127x8191": ("edge GEMM M=127 N=8191 K=2048 packed ld, alpha=0.5 beta=1, bf16 C in place", 1,
+                     127, 8191, 2048, "bf16", 0.5, 1.0, 1.0, 1.0, "normal", 3),
+    "recsys": ("batched shared-W GEMM Y[b]=W X[b], b<2048, W 256x512 N(0,1/sqrt(512)), X[b] 512x128 "
+               "N(0,1), bf16 out", 2048, 256, 128, 512, "bf16", 1.0, 0.0, 512 ** -0.5, 1.0, "normal", 4),
+}
+DEFAULT_WORKLOAD = "square8192"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "dsl_persistent_warp_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("kernel_source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def algorithmic_bytes(w) -> float:
+    _, batch, M, N, K, out, alpha, beta, *_ = w
+    es = 4 if out == "f32" else 2
+    a = M * K * 2  # W / A read once
+    b = batch * N * K * 2
+    c = batch * M * N * es * (2 if beta != 0.0 else 1)
+    return float(a + b + c)
+
+
+def launches_per_step(w) -> int:
+    """Kernels of this library one call enqueues: the GEMM, plus one alignment pre-pass copy per
+    operand whose leading dimension is not a multiple of 8 elements (packed ld here)."""
+    _, batch, M, N, K, *_ = w
+    n = 1
+    if K % 8:
+        n += 1  # A (lda = K)
+    if (N if batch > 1 else K) % 8:
+        n += 1  # B (ldb = K, or ldx = N for the batched form)
+    return n
+
+
+class ClockSampler(threading.Thread):
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+        "applications_clocks_setting": "nvmlClocksEventReasonApplicationsClocksSetting",
+        "sync_boost": "nvmlClocksEventReasonSyncBoost",
+    }
+
+    def __init__(self, torch_dev: int, period_s: float = 0.002):
+        super().__init__(daemon=True)
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            self.nv = pynvml
+            pynvml.nvmlInit()
+            p = torch.cuda.get_device_properties(torch_dev)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - reported in the JSON
+            self.err = repr(e)
+
+    def run(self):
+        if not self.ok:
+            return
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, const in self.REASONS.items():
+                    if mask & getattr(nv, const, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        self.join(timeout=2)
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        if not dist.is_initialized():
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def make_inputs(w, torch):
+    """Seeded synthetic inputs on the device (packed leading dimensions)."""
+    from synth import matrix_bf16, seed_for
+    desc, batch, M, N, K, out, alpha, beta, std_a, std_b, dist, idx = w
+
+    def dev(bits, shape):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).reshape(shape).cuda()
+
+    if batch == 1:
+        A = matrix_bf16(seed_for(idx, "A"), M, K, dist=dist, std=std_a)
+        B = matrix_bf16(seed_for(idx, "B"), N, K, dist=dist, std=std_b)
+        dA, dB = dev(A, (M, K)), dev(B, (N, K))
+        host = {"A": A, "B": B}
+    else:
+        A = matrix_bf16(seed_for(idx, "W"), M, K, dist=dist, std=std_a)
+        B = matrix_bf16(seed_for(idx, "X"), batch * K, N, dist=dist, std=std_b)
+        dA, dB = dev(A, (M, K)), dev(B, (batch, K, N))
+        host = {"A": A, "B": B}
+    odt = torch.float32 if out == "f32" else torch.bfloat16
+    shape = (M, N) if batch == 1 else (batch, M, N)
+    if beta != 0.0:
+        Cb = matrix_bf16(seed_for(idx, "C"), batch * M, N)
+        dC = dev(Cb, shape).to(odt)
+    else:
+        dC = torch.empty(shape, dtype=odt, device="cuda")
+    return dA, dB, dC, host
+
+
+def run_ours(args, w, wname):
+    import torch
+    import dsl_persistent_warp_b200 as pw
+
+    world, rank, local = dist_setup(args.gpus)
+    desc, batch, M, N, K, out, alpha, beta, *_ = w
+    flops = 2.0 * batch * M * N * K
+    dA, dB, dC, host = make_inputs(w, torch)
+
+    def step(C=dC):
+        if batch == 1:
+            pw.gemm_bf16(dA, dB, C, alpha=alpha, beta=beta)
+        else:
+            pw.gemm_bf16_batched_shared_w(dA, dB, C, alpha=alpha, beta=beta)
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if pw.device_status() != 0:
+        raise RuntimeError("kernel reported a bounded-wait timeout during warm-up")
+
+    sampler = ClockSampler(local)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(args.steps):
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    total_ms = starts[0].elapsed_time(ends[-1])
+    per_launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if pw.device_status() != 0:
+        raise RuntimeError("kernel reported a bounded-wait timeout in the timed region")
+    total_ms = max_over_ranks(total_ms, world)
+    value = flops * args.steps * world / (total_ms * 1e-3) / 1e12
+    avg_launch_ms = statistics.mean(per_launch_ms)
+
+    # end to end through the public API with host buffers: H2D of the inputs from pinned
+    # memory, the GEMM, D2H of the result, all inside the timed region.
+    hA = torch.from_numpy(host["A"].view(np.int16)).view(torch.bfloat16).reshape(dA.shape).pin_memory()
+    hB = torch.from_numpy(host["B"].view(np.int16)).view(torch.bfloat16).reshape(dB.shape).pin_memory()
+    hC = torch.empty(dC.shape, dtype=dC.dtype).pin_memory()
+    hC0 = dC.cpu().pin_memory() if beta != 0.0 else None
+    e2e_steps = max(1, min(args.steps, 10))
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        dA.copy_(hA, non_blocking=True)
+        dB.copy_(hB, non_blocking=True)
+        if hC0 is not None:
+            dC.copy_(hC0, non_blocking=True)
+        step()
+        hC.copy_(dC, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = hA.numel() * 2 + hB.numel() * 2 + (hC0.numel() * hC0.element_size() if hC0 is not None else 0)
+    d2h = hC.numel() * hC.element_size()
+    e2e_value = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, host, budget_s=args.cpu_seconds)
+
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (avg_launch_ms * 1e-3) / 1e12
+    traffic = recorded_traffic(wname)
+    res = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": desc,
+            "name": wname,
+            "batch": batch, "M": M, "N": N, "K": K,
+            "out": out, "alpha": alpha, "beta": beta,
+            "l2": "inputs larger than L2" if algorithmic_bytes(w) > L2_BYTES else
+                  "inputs smaller than L2 (steps back to back; no flush)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "pct_of_peak": {
+            "of_measured_burst": round(100.0 * value / world / peak, 2),
+            "of_spec_2250": round(100.0 * value / world / SPEC_BF16_TFLOPS, 2),
+            "peak_source": peak_kind,
+        },
+        "roofline": {
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "algorithmic_bytes": algorithmic_bytes(w),
+            "peak_kind": f"bf16 dense, burst ({peak_kind})",
+        },
+        "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
+        "gpu_launches": args.steps * launches_per_step(w),
+        "clocks": clocks,
+    }
+    if cpu is not None:
+        res["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def cpu_baseline(w, host, budget_s=15.0):
+    """The fp64 oracle, as it stands, on a bounded row sample of the same workload."""
+    import oracle
+    desc, batch, M, N, K, out, alpha, beta, *_ = w
+    A, B = host["A"], host["B"]
+
+    def run_rows(nrows):
+        rows = list(range(nrows))
+        t0 = time.perf_counter()
+        if batch == 1:
+            oracle.gemm(A, B, M=M, N=N, K=K, rows=rows)
+        else:
+            nb = max(1, nrows // M)
+            oracle.gemm_batched(A, B[: nb * K], batch=nb, M=M, N=N, K=K, stride_x=K * N)
+        return time.perf_counter() - t0
+
+    if batch == 1:
+        t = run_rows(min(M, 4))
+        per_row = max(t / min(M, 4), 1e-6)
+        nrows = int(max(1, min(M, budget_s / per_row)))
+        dt = run_rows(nrows)
+        flops = 2.0 * nrows * N * K
+        sample = f"{nrows} of {M} output rows (all {N} columns, full K={K})"
+    else:
+        t = run_rows(M)
+        nb = int(max(1, min(batch, budget_s / max(t, 1e-6))))
+        dt = run_rows(nb * M)
+        flops = 2.0 * nb * M * N * K
+        sample = f"{nb} of {batch} batches (full {M}x{N}x{K} each)"
+    return {"value": round(flops / dt / 1e12, 6), "unit": UNIT, "cores": oracle.threads(),
+            "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+
+
+def run_reference(args, w, wname):
+    """The fp64 CPU oracle timed on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from synth import matrix_bf16, seed_for
+    desc, batch, M, N, K, out, alpha, beta, std_a, std_b, dist, idx = w
+    # bounded sample: at most ~`ref_seconds` of CPU work over warmup + steps.
+    total_steps = args.steps + args.warmup
+    per_step_s = max(0.02, args.ref_seconds / max(total_steps, 1))
+    A = matrix_bf16(seed_for(idx, "A" if batch == 1 else "W"), M, K, dist=dist, std=std_a)
+    if batch == 1:
+        B = matrix_bf16(seed_for(idx, "B"), N, K, dist=dist, std=std_b)
+    else:
+        B = matrix_bf16(seed_for(idx, "X"), K, N, dist=dist, std=std_b)
+    c0 = matrix_bf16(seed_for(idx, "C"), M, N) if beta != 0.0 else None
+
+    def one(nrows):
+        rows = list(range(nrows))
+        if batch == 1:
+            oracle.gemm(A, B, M=M, N=N, K=K, c0=c0, alpha=alpha, beta=beta, rows=rows)
+        else:
+            oracle.gemm(A, B, M=M, N=N, K=K, b_kmajor=False, rows=rows)
+
+    t0 = time.perf_counter()
+    one(1)
+    per_row = max(time.perf_counter() - t0, 1e-6)
+    nrows = int(max(1, min(M, per_step_s / per_row)))
+    for _ in range(args.warmup):
+        one(nrows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one(nrows)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * nrows * N * K * args.steps
+    value = flops / dt / 1e12
+    sample = f"{nrows} of {M} output rows per step (all {N} columns, full K={K})" + (
+        f", one of {batch} batches" if batch > 1 else "")
+    res = {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": desc, "name": wname, "batch": batch, "M": M, "N": N, "K": K,
+                   "out": out, "alpha": alpha, "beta": beta, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(WORKLOADS) + ["all"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU seconds for the oracle baseline sample")
+    ap.add_argument("--ref-seconds", type=float, default=90.0,
+                    help="CPU seconds for the whole --impl reference run")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    names = sorted(WORKLOADS) if args.workload == "all" else [args.workload]
+    for n in names:
+        if args.impl == "reference":
+            run_reference(args, WORKLOADS[n], n)
+        else:
+            run_ours(args, WORKLOADS[n], n)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,401 @@
+// api.cu -- host side of the C ABI declared in include/gemm_bf16.h: argument validation,
+// tile-plan choice, tensor-map encoding, the alignment pre-pass and the kernel launches.
+// Every step of the computation runs in the kernels of gemm_kernel.cuh; this file only
+// prepares and enqueues them.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <array>
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "gemm_bf16.h"
+#include "gemm_kernel.cuh"
+
+using namespace pw;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+constexpr int kGroupM = 8;
+
+std::atomic<int> g_plan_override{-1};
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+struct DevInfo {
+    bool init = false;
+    int sms = 0;
+    int major = 0;
+    int minor = 0;
+};
+
+std::mutex g_dev_mu;
+std::array<DevInfo, kMaxDevices> g_dev;
+
+bool device_info(int dev, DevInfo& out) {
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo& d = g_dev[dev];
+    if (!d.init) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return false;
+        d.init = true;
+    }
+    out = d;
+    return true;
+}
+
+// One request, in the batched form (batch == 1 for the plain GEMM).
+struct Req {
+    int batch, M, N, K;
+    const void* A;
+    long long lda;
+    const void* B;
+    long long ldb, stride_b;
+    bool b_mn;  // B stored K x N (N-major) instead of N x K (K-major)
+    void* C;
+    long long ldc, stride_c;
+    int out;  // OUT_F32 / OUT_BF16
+    float alpha, beta;
+    cudaStream_t stream;
+};
+
+struct PlanDesc {
+    int cg, bn, stages;
+};
+constexpr PlanDesc kPlans[4] = {{1, 128, 6}, {1, 256, 4}, {2, 256, 6}, {2, 128, 8}};
+
+inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+inline long long round_up(long long a, long long b) { return cdiv(a, b) * b; }
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+gemm_status_t validate(const Req& r) {
+    if (r.batch < 0 || r.M < 0 || r.N < 0 || r.K < 0) return GEMM_ERR_INVALID_ARG;
+    if (r.out != OUT_F32 && r.out != OUT_BF16) return GEMM_ERR_INVALID_ARG;
+    const long long minA = r.K > 1 ? r.K : 1;
+    const long long minB = r.b_mn ? (r.N > 1 ? r.N : 1) : (r.K > 1 ? r.K : 1);
+    const long long minC = r.N > 1 ? r.N : 1;
+    if (r.lda < minA || r.ldb < minB || r.ldc < minC) return GEMM_ERR_INVALID_ARG;
+    if (r.stride_b < 0 || r.stride_c < 0) return GEMM_ERR_INVALID_ARG;
+    if (r.batch == 0 || r.M == 0 || r.N == 0) return GEMM_OK;
+    const uintptr_t es = r.out == OUT_F32 ? 4 : 2;
+    if (r.C == nullptr || !aligned(r.C, es)) return GEMM_ERR_INVALID_ARG;
+    if (r.batch > 1 && r.stride_c < (long long)(r.M - 1) * r.ldc + r.N) return GEMM_ERR_INVALID_ARG;
+    if (r.K > 0 && r.alpha != 0.0f) {
+        if (r.A == nullptr || r.B == nullptr) return GEMM_ERR_INVALID_ARG;
+        if (!aligned(r.A, 2) || !aligned(r.B, 2)) return GEMM_ERR_INVALID_ARG;
+    }
+    return GEMM_OK;
+}
+
+gemm_status_t encode_3d(CUtensorMap* m, const void* base, bool f32, uint64_t d0, uint64_t d1,
+                        uint64_t d2, uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return GEMM_ERR_CUDA;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {s1_bytes, s2_bytes};
+    cuuint32_t box[3] = {b0, b1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult res = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return res == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_CUDA;
+}
+
+// Plan for a request on a device with `sms` SMs (auto unless overridden).
+int choose_plan(const Req& r, int sms) {
+    const int forced = g_plan_override.load();
+    if (forced >= 0) return forced;
+    const long long t256x256 = cdiv(r.M, 256) * cdiv(r.N, 256) * r.batch;
+    const long long t256x128 = cdiv(r.M, 256) * cdiv(r.N, 128) * r.batch;
+    const long long t128x256 = cdiv(r.M, 128) * cdiv(r.N, 256) * r.batch;
+    if (t256x256 >= sms / 2) return 2;
+    if (t256x128 >= sms / 2) return 3;
+    if (t128x256 >= sms) return 1;
+    return 0;
+}
+
+template <int CG, int BN, int STAGES, int B_MN, int OUT>
+gemm_status_t launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
+                                const KParams& p, int dev, int sms, cudaStream_t stream) {
+    using T = Tile<CG, BN, STAGES, B_MN, OUT>;
+    auto kern = gemm_persistent<CG, BN, STAGES, B_MN, OUT>;
+    static std::array<std::atomic<int>, kMaxDevices> attr_done{};
+    static std::array<std::atomic<int>, kMaxDevices> max_clusters{};
+    if (!attr_done[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM_ALLOC) !=
+            cudaSuccess)
+            return GEMM_ERR_CUDA;
+        int clusters = sms / CG;
+        if constexpr (CG == 2) {
+            cudaLaunchConfig_t q = {};
+            q.gridDim = dim3(sms, 1, 1);
+            q.blockDim = dim3(T::THREADS, 1, 1);
+            q.dynamicSmemBytes = T::SMEM_ALLOC;
+            cudaLaunchAttribute qa[1];
+            qa[0].id = cudaLaunchAttributeClusterDimension;
+            qa[0].val.clusterDim.x = 2;
+            qa[0].val.clusterDim.y = 1;
+            qa[0].val.clusterDim.z = 1;
+            q.attrs = qa;
+            q.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &q) == cudaSuccess && n > 0 && n < clusters)
+                clusters = n;
+        }
+        max_clusters[dev].store(clusters);
+        attr_done[dev].store(1);
+    }
+    const int clusters = (int)(p.tiles < max_clusters[dev].load() ? p.tiles : max_clusters[dev].load());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(clusters * CG, 1, 1);
+    cfg.blockDim = dim3(T::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = T::SMEM_ALLOC;
+    cfg.stream = stream;
+    cudaLaunchAttribute attrs[1];
+    if constexpr (CG == 2) {
+        attrs[0].id = cudaLaunchAttributeClusterDimension;
+        attrs[0].val.clusterDim.x = 2;
+        attrs[0].val.clusterDim.y = 1;
+        attrs[0].val.clusterDim.z = 1;
+        cfg.attrs = attrs;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, p) == cudaSuccess ? GEMM_OK : GEMM_ERR_CUDA;
+}
+
+template <int CG, int BN, int STAGES>
+gemm_status_t launch_plan(bool b_mn, int out, const CUtensorMap& ma, const CUtensorMap& mb,
+                          const CUtensorMap& mc, const KParams& p, int dev, int sms, cudaStream_t st) {
+    if (b_mn) {
+        if constexpr ((BN / CG) % 64 == 0) {
+            return out == OUT_F32 ? launch_persistent<CG, BN, STAGES, 1, OUT_F32>(ma, mb, mc, p, dev, sms, st)
+                                  : launch_persistent<CG, BN, STAGES, 1, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
+        } else {
+            return GEMM_ERR_UNSUPPORTED;
+        }
+    }
+    return out == OUT_F32 ? launch_persistent<CG, BN, STAGES, 0, OUT_F32>(ma, mb, mc, p, dev, sms, st)
+                          : launch_persistent<CG, BN, STAGES, 0, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
+}
+
+gemm_status_t launch_scale(const Req& r) {
+    const long long total = (long long)r.batch * r.M * r.N;
+    const int threads = 256;
+    long long blocks = cdiv(total, threads);
+    if (blocks > 148LL * 32) blocks = 148LL * 32;
+    if (r.out == OUT_F32)
+        scale_c_kernel<float><<<(unsigned)blocks, threads, 0, r.stream>>>(
+            static_cast<float*>(r.C), r.ldc, r.stride_c, r.batch, r.M, r.N, r.beta);
+    else
+        scale_c_kernel<uint16_t><<<(unsigned)blocks, threads, 0, r.stream>>>(
+            static_cast<uint16_t*>(r.C), r.ldc, r.stride_c, r.batch, r.M, r.N, r.beta);
+    return cudaGetLastError() == cudaSuccess ? GEMM_OK : GEMM_ERR_CUDA;
+}
+
+void launch_pad(const void* src, long long ld_src, long long bs_src, void* dst, long long ld_dst,
+                long long bs_dst, int batch, int rows, int cols, cudaStream_t st) {
+    const int threads = 128;
+    int gx = (int)cdiv(cdiv(cols, 8), threads);
+    if (gx > 8) gx = 8;
+    int gy = rows < 4096 ? (rows > 0 ? rows : 1) : 4096;
+    int gz = batch < 65535 ? batch : 65535;
+    pad_copy_kernel<<<dim3(gx, gy, gz), threads, 0, st>>>(
+        static_cast<const uint16_t*>(src), ld_src, bs_src, static_cast<uint16_t*>(dst), ld_dst, bs_dst,
+        batch, rows, cols);
+}
+
+gemm_status_t run(Req r) {
+    gemm_status_t v = validate(r);
+    if (v != GEMM_OK) return v;
+    if (r.batch == 0 || r.M == 0 || r.N == 0) return GEMM_OK;
+    if (r.batch == 1) {
+        r.stride_b = r.b_mn ? (long long)r.K * r.ldb : (long long)r.N * r.ldb;
+        r.stride_c = (long long)r.M * r.ldc;
+    }
+    if (r.K == 0 || r.alpha == 0.0f) return launch_scale(r);
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GEMM_ERR_CUDA;
+    DevInfo di;
+    if (!device_info(dev, di)) return GEMM_ERR_CUDA;
+    if (di.major != 10 || di.minor != 0) return GEMM_ERR_UNSUPPORTED;
+
+    // Operands TMA cannot read as given go through a padded, 16-byte aligned copy.
+    const bool a_ok = aligned(r.A, 16) && (r.lda % 8) == 0;
+    const long long b_rows = r.b_mn ? r.K : r.N;  // rows of the stored B matrix per batch
+    const long long b_cols = r.b_mn ? r.N : r.K;
+    const bool b_ok = aligned(r.B, 16) && (r.ldb % 8) == 0 &&
+                      (r.batch == 1 || ((r.stride_b % 8) == 0 && r.stride_b >= b_rows * r.ldb));
+    long long lda_p = r.lda, ldb_p = r.ldb, sb_p = r.stride_b;
+    size_t ws_a = 0, ws_b = 0;
+    if (!a_ok) {
+        lda_p = round_up(r.K, 8);
+        ws_a = (size_t)round_up((long long)r.M * lda_p * 2, 256);
+    }
+    if (!b_ok) {
+        ldb_p = round_up(b_cols, 8);
+        sb_p = b_rows * ldb_p;
+        ws_b = (size_t)round_up(sb_p * 2 * r.batch, 256);
+    }
+    void* ws = nullptr;
+    if (ws_a + ws_b) {
+        if (cudaMallocAsync(&ws, ws_a + ws_b, r.stream) != cudaSuccess) return GEMM_ERR_NO_MEMORY;
+    }
+    const void* A = r.A;
+    const void* B = r.B;
+    if (!a_ok) {
+        launch_pad(r.A, r.lda, 0, ws, lda_p, 0, 1, r.M, r.K, r.stream);
+        A = ws;
+    }
+    if (!b_ok) {
+        void* dst = static_cast<char*>(ws) + ws_a;
+        launch_pad(r.B, r.ldb, r.stride_b, dst, ldb_p, sb_p, r.batch, (int)b_rows, (int)b_cols, r.stream);
+        B = dst;
+    }
+
+    const int plan = choose_plan(r, di.sms);
+    const PlanDesc pd = kPlans[plan];
+    const int bn_cta = pd.bn / pd.cg;
+    const int es = r.out == OUT_F32 ? 4 : 2;
+    const int stg_cols = r.out == OUT_F32 ? 32 : 64;
+    const bool c_tma = aligned(r.C, 16) && ((r.ldc * es) % 16) == 0 &&
+                       (r.batch == 1 || ((r.stride_c * es) % 16) == 0);
+
+    CUtensorMap ma, mb, mc;
+    std::memset(&mc, 0, sizeof mc);
+    gemm_status_t st = encode_3d(&ma, A, false, (uint64_t)r.K, (uint64_t)r.M, 1, (uint64_t)lda_p * 2,
+                                 (uint64_t)lda_p * 2 * (uint64_t)r.M, 64, 128);
+    if (st == GEMM_OK) {
+        if (!r.b_mn)
+            st = encode_3d(&mb, B, false, (uint64_t)r.K, (uint64_t)r.N, (uint64_t)r.batch,
+                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, 64, (uint32_t)bn_cta);
+        else
+            st = encode_3d(&mb, B, false, (uint64_t)r.N, (uint64_t)r.K, (uint64_t)r.batch,
+                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, 64, 64);
+    }
+    if (st == GEMM_OK && c_tma)
+        st = encode_3d(&mc, r.C, r.out == OUT_F32, (uint64_t)r.N, (uint64_t)r.M, (uint64_t)r.batch,
+                       (uint64_t)r.ldc * es, (uint64_t)r.stride_c * es, (uint32_t)stg_cols, 32);
+    if (st == GEMM_OK) {
+        KParams p;
+        std::memset(&p, 0, sizeof p);
+        p.M = r.M;
+        p.N = r.N;
+        p.K = r.K;
+        p.m_blocks = (int)cdiv(r.M, 128 * pd.cg);
+        p.n_blocks = (int)cdiv(r.N, pd.bn);
+        p.batch = r.batch;
+        p.tiles = p.m_blocks * p.n_blocks * r.batch;
+        p.k_blocks = (int)cdiv(r.K, 64);
+        p.group_m = kGroupM;
+        p.alpha = r.alpha;
+        p.beta = r.beta;
+        p.C = r.C;
+        p.ldc = r.ldc;
+        p.stride_c = r.stride_c;
+        p.c_tma = c_tma ? 1 : 0;
+        p.c_read = r.beta != 0.0f ? 1 : 0;
+        p.timeout_ns = g_timeout_ns.load();
+        switch (plan) {
+            case 0: st = launch_plan<1, 128, 6>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream); break;
+            case 1: st = launch_plan<1, 256, 4>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream); break;
+            case 2: st = launch_plan<2, 256, 6>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream); break;
+            default: st = launch_plan<2, 128, 8>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream); break;
+        }
+    }
+    if (ws) cudaFreeAsync(ws, r.stream);
+    return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+gemm_status_t gemm_bf16(int M, int N, int K, const void* A, int lda, const void* B, int ldb, void* C,
+                        int ldc, gemm_out_t out_type, float alpha, float beta, cudaStream_t stream) {
+    try {
+        Req r{1, M, N, K, A, lda, B, ldb, 0, false, C, ldc, 0, (int)out_type, alpha, beta, stream};
+        return run(r);
+    } catch (...) {
+        return GEMM_ERR_CUDA;
+    }
+}
+
+gemm_status_t gemm_bf16_batched_shared_w(int batch, int M, int N, int K, const void* W, int ldw,
+                                         const void* X, int ldx, long long stride_x, void* Y, int ldy,
+                                         long long stride_y, gemm_out_t out_type, float alpha,
+                                         float beta, cudaStream_t stream) {
+    try {
+        Req r{batch, M, N, K, W, ldw, X, ldx, stride_x, true, Y, ldy, stride_y, (int)out_type,
+              alpha, beta, stream};
+        return run(r);
+    } catch (...) {
+        return GEMM_ERR_CUDA;
+    }
+}
+
+const char* gemm_bf16_status_string(gemm_status_t s) {
+    switch (s) {
+        case GEMM_OK: return "GEMM_OK";
+        case GEMM_ERR_INVALID_ARG: return "GEMM_ERR_INVALID_ARG";
+        case GEMM_ERR_UNSUPPORTED: return "GEMM_ERR_UNSUPPORTED";
+        case GEMM_ERR_CUDA: return "GEMM_ERR_CUDA";
+        case GEMM_ERR_TIMEOUT: return "GEMM_ERR_TIMEOUT";
+        case GEMM_ERR_NO_MEMORY: return "GEMM_ERR_NO_MEMORY";
+    }
+    return "GEMM_ERR_UNKNOWN";
+}
+
+gemm_status_t gemm_bf16_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GEMM_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_pw_status, sizeof v) != cudaSuccess) return GEMM_ERR_CUDA;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_pw_status, &zero, sizeof zero) != cudaSuccess) return GEMM_ERR_CUDA;
+        return GEMM_ERR_TIMEOUT;
+    }
+    return GEMM_OK;
+}
+
+gemm_status_t gemm_bf16_set_plan(int plan) {
+    if (plan < -1 || plan > 3) return GEMM_ERR_INVALID_ARG;
+    g_plan_override.store(plan);
+    return GEMM_OK;
+}
+
+gemm_status_t gemm_bf16_set_wait_timeout_ns(unsigned long long ns) {
+    g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
+    return GEMM_OK;
+}
+
+int gemm_bf16_version(void) { return 100; }
+
+}  // extern "C"

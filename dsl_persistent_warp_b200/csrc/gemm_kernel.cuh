@@ -1,0 +1,501 @@
+// gemm_kernel.cuh -- the persistent, warp-specialized BF16 GEMM for sm_100a.
+//
+// Computes C = alpha * A * B + beta * C (bf16 in, fp32 accumulate) over a grid of output
+// tiles, following the producer/consumer structure described for TLX on the page
+// "Meta presente TLX pour combler le fosse entre la complexite du materiel GPU et la
+// productivite des developpeurs", section "Comment cela fonctionne": one warp loads tiles
+// asynchronously through TMA while another drives the tensor cores, and lightweight
+// barriers (mbarriers) hand each stage over, giving a deep pipeline that overlaps data
+// movement and math.  The multi-stage shared-memory ring and the K loop over staged tiles
+// correspond to the Hopper sketch on the page "Triton 3.7 permite extender el compilador de
+// GPU sin forks", section "NVIDIA H100 (Hopper): GEMM persistente" (NUM_STAGES buffers,
+// prefetch ahead, accumulate, store); the grouped tile order is its GROUP_SIZE_M parameter.
+//
+// Blackwell design (not from the pages):
+//   * warp 0, one lane      : TMA producer.  Waits empty[s], arms full[s] with the stage's
+//                             byte count, issues the A and B tile loads (no multicast).
+//   * warp 1, one lane      : MMA issuer (leader CTA only).  Waits full[s], issues
+//                             tcgen05.mma (K=16 per instruction) into a TMEM accumulator,
+//                             commits empty[s]; after the last k-block commits tmem_full.
+//   * warps 2..5            : epilogue.  Wait tmem_full, tcgen05.ld 32 rows x 32 columns per
+//                             warp, release the accumulator (tmem_empty), apply alpha/beta,
+//                             convert, stage through swizzled shared memory and TMA-store.
+//   * two TMEM accumulators : the epilogue of tile i overlaps the mainloop of tile i+1.
+//   * CG = 2                : a 2-CTA cluster computes a 256-row tile with
+//                             tcgen05.mma.cta_group::2; each CTA loads its 128 rows of A and
+//                             half of the tile's B columns; loads of both CTAs complete on the
+//                             leader's full barrier, commits go to both CTAs' barriers.
+//   * every barrier wait is bounded (global timer); on expiry the kernel records a status
+//     bit, raises an abort flag, lets in-flight copies land, frees TMEM and returns.
+#pragma once
+#include <cuda.h>
+#include <cstdint>
+
+#include "ptx_sm100.cuh"
+
+namespace pw {
+
+enum : int { OUT_F32 = 0, OUT_BF16 = 1 };
+
+// Device status word: bit i set = a bounded wait of role i expired (see kStatus*).
+__device__ unsigned int g_pw_status;
+
+enum : unsigned int {
+    kStatusProducer = 1u,
+    kStatusMma = 2u,
+    kStatusEpilogue = 4u,
+};
+
+struct KParams {
+    int M, N, K;
+    int m_blocks, n_blocks;  // cluster tiles along M and N
+    int batch;
+    int tiles;               // batch * m_blocks * n_blocks
+    int k_blocks;            // ceil(K / 64)
+    int group_m;             // grouped raster: m-blocks per group
+    float alpha, beta;
+    void* C;                 // output base (also the beta input)
+    long long ldc;           // elements
+    long long stride_c;      // elements between batches of C
+    int c_tma;               // 1: epilogue uses TMA stores (aligned C), 0: direct stores
+    int c_read;              // 1: beta != 0
+    unsigned long long timeout_ns;
+};
+
+template <int CG, int BN, int STAGES, int B_MN, int OUT>
+struct Tile {
+    static constexpr int BK = 64;                   // K per stage (128 B of bf16)
+    static constexpr int BM = 128 * CG;             // rows of the cluster tile (MMA M)
+    static constexpr int BN_CTA = BN / CG;          // B rows (N) loaded by each CTA
+    static constexpr int A_BYTES = 128 * BK * 2;
+    static constexpr int B_BYTES = BN_CTA * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int EPI_WARPS = 4;
+    static constexpr int THREADS = 32 * (2 + EPI_WARPS);
+    static constexpr int STG_COLS = OUT == OUT_F32 ? 32 : 64;  // 128-byte rows
+    static constexpr int STG_BYTES = 32 * 128;
+    static constexpr int CHUNKS = BN / STG_COLS;
+    static constexpr int TMEM_COLS = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128
+                                   : 2 * BN <= 256 ? 256 : 512;
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * 2 * STG_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 4;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16;
+    static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack to align the base to 1 KiB
+    static_assert(BN % (16 * CG) == 0 && BN <= 256, "MMA N");
+    static_assert(!B_MN || BN_CTA % 64 == 0, "MN-major B is loaded in 64-column boxes");
+    static_assert(BN % STG_COLS == 0, "epilogue chunks");
+    static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
+};
+
+// Tile t -> (batch, m-block, n-block); m-blocks are walked in groups of group_m so that
+// the CTAs resident at one time share A and B panels in L2.
+__device__ __forceinline__ void decode_tile(const KParams& p, int t, int& b, int& mb, int& nb) {
+    const int per_batch = p.m_blocks * p.n_blocks;
+    b = t / per_batch;
+    const int r = t - b * per_batch;
+    const int group_size = p.group_m * p.n_blocks;
+    const int g = r / group_size;
+    const int first_m = g * p.group_m;
+    const int gm = min(p.m_blocks - first_m, p.group_m);
+    const int w = r - g * group_size;
+    mb = first_m + w % gm;
+    nb = w / gm;
+}
+
+template <int CG>
+__device__ __forceinline__ void raise_abort(uint32_t slot_abort, uint32_t rank, unsigned int code) {
+    atomicOr(&g_pw_status, code);
+    st_shared_volatile_u32(slot_abort, 1u);
+    if constexpr (CG == 2) st_cluster_u32(map_to_rank(slot_abort, rank ^ 1u), 1u);
+}
+
+// Bounded wait on an mbarrier phase.  Returns false when the kernel is aborting (this wait
+// expired, or another role raised the abort flag).
+template <int CG, bool CLUSTER_SCOPE>
+__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint32_t slot_abort,
+                                        uint32_t rank, unsigned long long timeout_ns,
+                                        unsigned int code) {
+    if (CLUSTER_SCOPE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i)
+            if (CLUSTER_SCOPE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity))
+                return true;
+        if (ld_shared_volatile_u32(slot_abort) != 0u) return false;
+        if (global_timer_ns() - t0 > timeout_ns) {
+            raise_abort<CG>(slot_abort, rank, code);
+            return false;
+        }
+    }
+}
+
+template <int CG, int BN, int STAGES, int B_MN, int OUT>
+__global__ void __launch_bounds__(Tile<CG, BN, STAGES, B_MN, OUT>::THREADS, 1)
+    gemm_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmC, const KParams p) {
+    using T = Tile<CG, BN, STAGES, B_MN, OUT>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (sbase - raw);
+
+    const uint32_t warp = threadIdx.x >> 5;
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+    const int cluster_id = blockIdx.x / CG;
+    const int num_clusters = gridDim.x / CG;
+
+    const uint32_t bar0 = sbase + T::OFF_BAR;
+    auto bar_full = [&](int s) { return bar0 + 8u * s; };
+    auto bar_empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto bar_tfull = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+    auto bar_tempty = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+    const uint32_t slot_tmem = sbase + T::OFF_MISC;
+    const uint32_t slot_abort = sbase + T::OFF_MISC + 4;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_empty(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(bar_tfull(a), 1);
+            mbar_init(bar_tempty(a), T::EPI_WARPS * CG);
+        }
+        st_shared_volatile_u32(slot_abort, 0u);
+        fence_mbarrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        if (p.c_tma) tma_prefetch_desc(&tmC);
+    }
+    if (warp == 1) {
+        tmem_alloc<CG>(slot_tmem, T::TMEM_COLS);
+        tmem_relinquish<CG>();
+    }
+    tc_fence_before();
+    if constexpr (CG == 2) cluster_sync(); else __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + T::OFF_MISC);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_normal();
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int t = cluster_id; t < p.tiles; t += num_clusters) {
+                int b, mb, nb;
+                decode_tile(p, t, b, mb, nb);
+                const int a_row = mb * T::BM + (int)rank * 128;
+                const int b_row = nb * BN + (int)rank * T::BN_CTA;
+                bool ok = true;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!wait_phase<CG, false>(bar_empty(stage), phase ^ 1u, slot_abort, rank,
+                                               p.timeout_ns, kStatusProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full_local = bar_full(stage);
+                    if (rank == 0) mbar_arrive_expect_tx(full_local, T::STAGE_BYTES * CG);
+                    const uint32_t sa = sbase + T::OFF_A + stage * T::A_BYTES;
+                    const uint32_t sb = sbase + T::OFF_B + stage * T::B_BYTES;
+                    const int k0 = kb * T::BK;
+                    if constexpr (CG == 1) {
+                        tma_load_3d(sa, &tmA, full_local, k0, a_row, 0, pol);
+                        if constexpr (!B_MN) {
+                            tma_load_3d(sb, &tmB, full_local, k0, b_row, b, pol);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < T::BN_CTA / 64; ++j)
+                                tma_load_3d(sb + j * 8192, &tmB, full_local, b_row + 64 * j, k0, b, pol);
+                        }
+                    } else {
+                        const uint32_t full_leader = map_to_rank(full_local, 0);
+                        tma_load_3d_pair(sa, &tmA, full_leader, k0, a_row, 0, pol);
+                        if constexpr (!B_MN) {
+                            tma_load_3d_pair(sb, &tmB, full_leader, k0, b_row, b, pol);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < T::BN_CTA / 64; ++j)
+                                tma_load_3d_pair(sb + j * 8192, &tmB, full_leader, b_row + 64 * j, k0, b,
+                                                 pol);
+                        }
+                    }
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t IDESC = idesc_bf16_f32(T::BM, BN, 0, B_MN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int t = cluster_id; t < p.tiles; t += num_clusters) {
+                if (!wait_phase<CG, CG == 2>(bar_tempty(acc), acc_phase ^ 1u, slot_abort, rank,
+                                             p.timeout_ns, kStatusMma))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                bool ok = true;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, rank, p.timeout_ns,
+                                               kStatusMma)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = sbase + T::OFF_A + stage * T::A_BYTES;
+                    const uint32_t sb = sbase + T::OFF_B + stage * T::B_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < T::BK / 16; ++kk) {
+                        const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
+                        const uint64_t bdesc = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                                    : smem_desc_sw128(sb + kk * 32, 16, 1024);
+                        umma_f16<CG>(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    if constexpr (CG == 1) {
+                        umma_commit<1>(bar_empty(stage));
+                    } else {
+                        umma_commit<2>(map_to_rank(bar_empty(stage), 0));
+                        umma_commit<2>(map_to_rank(bar_empty(stage), 1));
+                    }
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                if constexpr (CG == 1) {
+                    umma_commit<1>(bar_tfull(acc));
+                } else {
+                    umma_commit<2>(map_to_rank(bar_tfull(acc), 0));
+                    umma_commit<2>(map_to_rank(bar_tfull(acc), 1));
+                }
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = (int)warp - 2;       // 0..3
+        const int q = (int)(warp & 3u);     // TMEM lane quarter this warp may access
+        const uint32_t stg = sbase + T::OFF_STG + ew * 2 * T::STG_BYTES;
+        constexpr int ES = OUT == OUT_F32 ? 4 : 2;
+        const uint32_t tempty_leader0 = CG == 2 ? map_to_rank(bar_tempty(0), 0) : bar_tempty(0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int buf = 0;
+        for (int t = cluster_id; t < p.tiles; t += num_clusters) {
+            int b, mb, nb;
+            decode_tile(p, t, b, mb, nb);
+            const int row0 = mb * T::BM + (int)rank * 128 + 32 * q;
+            const int row = row0 + (int)lane;
+            const int col0 = nb * BN;
+            int ok = 1;
+            if (lane == 0)
+                ok = wait_phase<CG, false>(bar_tfull(acc), acc_phase, slot_abort, rank, p.timeout_ns,
+                                           kStatusEpilogue);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
+            const long long cbase = (long long)b * p.stride_c + (long long)row * p.ldc;
+#pragma unroll 1
+            for (int c = 0; c < T::CHUNKS; ++c) {
+                float v[T::STG_COLS];
+                {
+                    uint32_t r0[32];
+                    tmem_ld_32x32b_x32(trow + c * T::STG_COLS, r0);
+                    if constexpr (OUT == OUT_BF16) {
+                        uint32_t r1[32];
+                        tmem_ld_32x32b_x32(trow + c * T::STG_COLS + 32, r1);
+                        tmem_ld_wait(r0);
+                        tmem_ld_wait(r1);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[32 + j] = __uint_as_float(r1[j]);
+                    } else {
+                        tmem_ld_wait(r0);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
+                }
+                if (c == T::CHUNKS - 1) {
+                    // Accumulator drained: hand it back to the MMA warp (leader CTA).
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * acc);
+                }
+                const int colc = col0 + c * T::STG_COLS;
+                const bool row_in = row < p.M;
+                const bool full_cols = colc + T::STG_COLS <= p.N;
+#pragma unroll
+                for (int j = 0; j < T::STG_COLS; ++j) v[j] *= p.alpha;
+                if (p.c_read && row_in) {
+                    if (full_cols && p.c_tma) {
+                        if constexpr (OUT == OUT_BF16) {
+                            const uint4* src = reinterpret_cast<const uint4*>(
+                                static_cast<const uint16_t*>(p.C) + cbase + colc);
+#pragma unroll
+                            for (int j = 0; j < T::STG_COLS / 8; ++j) {
+                                const uint4 w = src[j];
+                                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                                for (int h = 0; h < 4; ++h) {
+                                    v[8 * j + 2 * h] = fmaf(p.beta, __uint_as_float(ww[h] << 16), v[8 * j + 2 * h]);
+                                    v[8 * j + 2 * h + 1] =
+                                        fmaf(p.beta, __uint_as_float(ww[h] & 0xFFFF0000u), v[8 * j + 2 * h + 1]);
+                                }
+                            }
+                        } else {
+                            const float4* src = reinterpret_cast<const float4*>(
+                                static_cast<const float*>(p.C) + cbase + colc);
+#pragma unroll
+                            for (int j = 0; j < T::STG_COLS / 4; ++j) {
+                                const float4 w = src[j];
+                                v[4 * j + 0] = fmaf(p.beta, w.x, v[4 * j + 0]);
+                                v[4 * j + 1] = fmaf(p.beta, w.y, v[4 * j + 1]);
+                                v[4 * j + 2] = fmaf(p.beta, w.z, v[4 * j + 2]);
+                                v[4 * j + 3] = fmaf(p.beta, w.w, v[4 * j + 3]);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < T::STG_COLS; ++j) {
+                            if (colc + j < p.N) {
+                                float cin;
+                                if constexpr (OUT == OUT_BF16)
+                                    cin = __uint_as_float((uint32_t)(static_cast<const uint16_t*>(p.C)[cbase + colc + j]) << 16);
+                                else
+                                    cin = static_cast<const float*>(p.C)[cbase + colc + j];
+                                v[j] = fmaf(p.beta, cin, v[j]);
+                            }
+                        }
+                    }
+                }
+                // pack the 128-byte row segment into 8 x 16-byte words
+                uint32_t w[32];
+                if constexpr (OUT == OUT_BF16) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
+                }
+                if (p.c_tma) {
+                    const uint32_t sb = stg + buf * T::STG_BYTES;
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                    const uint32_t row_addr = sb + lane * 128u;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        st_shared_v4(row_addr + ((uint32_t)(j ^ (int)(lane & 7u)) << 4), w[4 * j],
+                                     w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tmC, sb, colc, row0, b);
+                        bulk_commit_group();
+                    }
+                    buf ^= 1;
+                } else if (row_in) {
+                    if constexpr (OUT == OUT_BF16) {
+                        uint16_t* dst = static_cast<uint16_t*>(p.C) + cbase + colc;
+#pragma unroll
+                        for (int j = 0; j < T::STG_COLS; ++j)
+                            if (colc + j < p.N)
+                                dst[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
+                    } else {
+                        float* dst = static_cast<float*>(p.C) + cbase + colc;
+#pragma unroll
+                        for (int j = 0; j < T::STG_COLS; ++j)
+                            if (colc + j < p.N) dst[j] = __uint_as_float(w[j]);
+                    }
+                }
+                (void)ES;
+            }
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+        if (p.c_tma && lane == 0) bulk_wait_group_all();
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (ld_shared_volatile_u32(slot_abort) != 0u && threadIdx.x == 0) {
+        // Aborting: let copies and MMAs already issued by this CTA land (bounded).
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 5000000ull) nanosleep_ns(100000);
+    }
+    if constexpr (CG == 2) cluster_sync(); else __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc<CG>(tmem_base, T::TMEM_COLS);
+    }
+}
+
+// C = beta * C (C = 0 when beta == 0) over batch x M x N: the K == 0 / alpha == 0 case.
+template <typename TC>
+__global__ void scale_c_kernel(TC* C, long long ldc, long long stride_c, int batch, int M, int N,
+                               float beta) {
+    const long long per = (long long)M * N;
+    const long long total = per * batch;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long b = i / per;
+        const long long r = (i - b * per) / N;
+        const long long c = i - b * per - r * N;
+        TC* e = C + b * stride_c + r * ldc + c;
+        float x = 0.0f;
+        if constexpr (sizeof(TC) == 2) {
+            if (beta != 0.0f) x = beta * __uint_as_float((uint32_t)(*reinterpret_cast<uint16_t*>(e)) << 16);
+            *reinterpret_cast<uint16_t*>(e) = (uint16_t)(pack_bf16x2(x, 0.0f) & 0xFFFFu);
+        } else {
+            if (beta != 0.0f) x = beta * *reinterpret_cast<float*>(e);
+            *reinterpret_cast<float*>(e) = x;
+        }
+    }
+}
+
+// Copy a batch x rows x cols bf16 array into a buffer whose leading dimension is a multiple
+// of 8 elements and whose base is 16-byte aligned, so that TMA can read it.
+__global__ void pad_copy_kernel(const uint16_t* __restrict__ src, long long ld_src, long long bs_src,
+                                uint16_t* __restrict__ dst, long long ld_dst, long long bs_dst,
+                                int batch, int rows, int cols) {
+    const int vec_per_row = (cols + 7) >> 3;
+    for (int b = blockIdx.z; b < batch; b += gridDim.z) {
+        for (int r = blockIdx.y; r < rows; r += gridDim.y) {
+            const uint16_t* s = src + b * bs_src + (long long)r * ld_src;
+            uint16_t* d = dst + b * bs_dst + (long long)r * ld_dst;
+            for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vec_per_row;
+                 v += gridDim.x * blockDim.x) {
+                const int c = v << 3;
+                if (c + 8 <= cols) {
+                    uint32_t e[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        e[j] = (uint32_t)s[c + 2 * j] | ((uint32_t)s[c + 2 * j + 1] << 16);
+                    *reinterpret_cast<uint4*>(d + c) = make_uint4(e[0], e[1], e[2], e[3]);
+                } else {
+                    for (int j = c; j < cols; ++j) d[j] = s[j];
+                }
+            }
+        }
+    }
+}
+
+}  // namespace pw

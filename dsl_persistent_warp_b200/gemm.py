@@ -1,0 +1,89 @@
+"""PyTorch-facing wrappers of the C ABI: torch supplies device memory, pointers, strides and the
+current stream; every step of the computation runs in the library's kernels.
+
+    C = alpha * A @ B_stored.T + beta * C          gemm_bf16(A, B_stored, C)
+    Y[b] = alpha * W @ X[b] + beta * Y[b]          gemm_bf16_batched_shared_w(W, X, Y)
+"""
+from __future__ import annotations
+
+import torch
+
+from . import capi
+
+_OUT = {torch.float32: capi.GEMM_OUT_F32, torch.bfloat16: capi.GEMM_OUT_BF16}
+
+
+def _stream_handle(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != capi.GEMM_OK:
+        raise capi.GemmError(status, what)
+
+
+def _rowmajor_2d(t: torch.Tensor, name: str):
+    if t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+        raise ValueError(f"{name} must be a 2-D row-major tensor (unit column stride)")
+    return max(int(t.stride(0)), 1) if t.shape[0] > 1 else max(int(t.shape[1]), 1)
+
+
+def gemm_bf16(A: torch.Tensor, B: torch.Tensor, C: torch.Tensor | None = None, *, alpha: float = 1.0,
+              beta: float = 0.0, out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+    """C = alpha * A @ B.T + beta * C for A (M x K) and B stored N x K ("K-major"), both bf16
+    CUDA tensors with unit column stride.  C (M x N, float32 or bfloat16) is updated in place
+    and returned; when omitted it is allocated (beta must then be 0)."""
+    if A.dtype != torch.bfloat16 or B.dtype != torch.bfloat16:
+        raise TypeError("A and B must be bfloat16")
+    M, K = A.shape
+    N, K2 = B.shape
+    if K2 != K:
+        raise ValueError("A and B disagree on K")
+    if C is None:
+        if beta != 0.0:
+            raise ValueError("beta != 0 needs C")
+        C = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    if C.shape != (M, N) or C.dtype not in _OUT:
+        raise ValueError("C must be M x N float32/bfloat16")
+    lda = _rowmajor_2d(A, "A") if K else 1
+    ldb = _rowmajor_2d(B, "B") if K else 1
+    ldc = _rowmajor_2d(C, "C")
+    st = capi.gemm_bf16(M, N, K, A.data_ptr(), max(lda, K, 1), B.data_ptr(), max(ldb, K, 1),
+                        C.data_ptr(), max(ldc, N, 1), _OUT[C.dtype], float(alpha), float(beta),
+                        _stream_handle(stream))
+    _check(st, "gemm_bf16")
+    return C
+
+
+def gemm_bf16_batched_shared_w(W: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = None, *,
+                               alpha: float = 1.0, beta: float = 0.0,
+                               out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+    """Y[b] = alpha * W @ X[b] + beta * Y[b] for W (M x K, shared), X (batch x K x N) and
+    Y (batch x M x N), all with unit innermost stride."""
+    if W.dtype != torch.bfloat16 or X.dtype != torch.bfloat16:
+        raise TypeError("W and X must be bfloat16")
+    M, K = W.shape
+    batch, K2, N = X.shape
+    if K2 != K:
+        raise ValueError("W and X disagree on K")
+    if Y is None:
+        if beta != 0.0:
+            raise ValueError("beta != 0 needs Y")
+        Y = torch.empty((batch, M, N), dtype=out_dtype, device=W.device)
+    if Y.shape != (batch, M, N) or Y.dtype not in _OUT:
+        raise ValueError("Y must be batch x M x N float32/bfloat16")
+    if (N > 1 and X.stride(2) != 1) or (N > 1 and Y.stride(2) != 1):
+        raise ValueError("X and Y need unit innermost stride")
+    ldw = _rowmajor_2d(W, "W") if K else 1
+    st = capi.gemm_bf16_batched_shared_w(
+        batch, M, N, K, W.data_ptr(), max(ldw, K, 1), X.data_ptr(), max(int(X.stride(1)), N, 1),
+        int(X.stride(0)), Y.data_ptr(), max(int(Y.stride(1)), N, 1), int(Y.stride(0)), _OUT[Y.dtype],
+        float(alpha), float(beta), _stream_handle(stream))
+    _check(st, "gemm_bf16_batched_shared_w")
+    return Y
+
+
+def device_status(stream=None) -> int:
+    """Synchronize the stream and return the library's device status (GEMM_OK / TIMEOUT)."""
+    return capi.gemm_bf16_device_status(_stream_handle(stream))

@@ -1,0 +1,135 @@
+/*
+ * gemm_bf16.h -- C ABI of the B200 (sm_100a) persistent, warp-specialized BF16 GEMM.
+ *
+ * The operation is the producer/consumer matrix multiply described on the page
+ * "Meta presente TLX pour combler le fosse entre la complexite du materiel GPU et la
+ * productivite des developpeurs", section "Comment cela fonctionne" (one warp group loads
+ * tiles asynchronously through TMA while another drives the tensor cores, handing over
+ * through lightweight barriers), whose accumulator loop is sketched on the page
+ * "Triton 3.7 permite extender el compilador de GPU sin forks", section "NVIDIA H100
+ * (Hopper): GEMM persistente" (fp32 accumulator, K loop over staged tiles, results stored),
+ * with the alpha/beta update of a BLAS GEMM:
+ *
+ *     C = alpha * A * B + beta * C       bf16 inputs, fp32 accumulation.
+ *
+ * All matrices are row-major in device memory; leading dimensions and strides are in
+ * ELEMENTS.  Calls are asynchronous: they validate the arguments, enqueue the kernels on
+ * `stream` and return.  The caller owns every buffer it passes; the library never frees
+ * them.  The library owns only a stream-ordered workspace (taken from the device's default
+ * memory pool with cudaMallocAsync and released with cudaFreeAsync on `stream`) that is
+ * used when A or B cannot be read by the tensor-memory accelerator as given (a leading
+ * dimension that is not a multiple of 8 elements, a base not 16-byte aligned).
+ *
+ * No exceptions cross this boundary.  Nothing is enqueued when a call returns an error.
+ */
+#ifndef GEMM_BF16_H
+#define GEMM_BF16_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GEMM_API __attribute__((visibility("default")))
+#else
+#define GEMM_API
+#endif
+
+struct CUstream_st; /* cudaStream_t == struct CUstream_st*; NULL is the legacy stream */
+
+typedef enum {
+    GEMM_OK = 0,
+    GEMM_ERR_INVALID_ARG = 1, /* bad size, leading dimension, pointer or enum */
+    GEMM_ERR_UNSUPPORTED = 2, /* valid request this build cannot run (e.g. no sm_100 GPU) */
+    GEMM_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (launch, encode, alloc) */
+    GEMM_ERR_TIMEOUT = 4,     /* a kernel gave up a bounded wait (see gemm_bf16_device_status) */
+    GEMM_ERR_NO_MEMORY = 5    /* the workspace allocation failed */
+} gemm_status_t;
+
+typedef enum {
+    GEMM_OUT_F32 = 0, /* C is float32 */
+    GEMM_OUT_BF16 = 1 /* C is bfloat16 (fp32 result rounded to nearest even once) */
+} gemm_out_t;
+
+/*
+ * gemm_bf16 -- C[M x N] = alpha * A[M x K] * B + beta * C.
+ *
+ *   A   bf16, M x K row-major, element (i,k) at A[i*lda + k], lda >= max(1, K).
+ *   B   bf16, stored N x K row-major ("K-major"), element (k,j) of the K x N operand at
+ *       B[j*ldb + k], ldb >= max(1, K).  So C = alpha * A * B_stored^T + beta * C.
+ *   C   out_type, M x N row-major, element (i,j) at C[i*ldc + j], ldc >= max(1, N).
+ *       Read only when beta != 0 (so NaN/garbage in C is ignored when beta == 0) and
+ *       updated in place.  Elements of the ldc padding columns are never touched.
+ *   alpha, beta  fp32 scalars.  D = alpha*acc + beta*C_in is formed in fp32 and, for
+ *       bf16 output, rounded once to nearest even.
+ *
+ * M == 0 or N == 0: returns GEMM_OK with nothing enqueued.  K == 0 or alpha == 0:
+ * C = beta * C (C = 0 when beta == 0) without reading A or B.
+ * Errors: GEMM_ERR_INVALID_ARG for negative sizes, a leading dimension below its minimum,
+ * a NULL pointer where data is needed, a pointer not aligned to its element size, or an
+ * unknown out_type.  A or B overlapping C is undefined behaviour (not checked).
+ * Results are deterministic: the same inputs give bitwise the same C on every call.
+ */
+GEMM_API gemm_status_t gemm_bf16(int M, int N, int K, const void* A, int lda, const void* B, int ldb,
+                        void* C, int ldc, gemm_out_t out_type, float alpha, float beta,
+                        struct CUstream_st* stream);
+
+/*
+ * gemm_bf16_batched_shared_w -- Y[b] = alpha * W * X[b] + beta * Y[b] for b < batch.
+ *
+ * The shared-operand form of the recommendation-model "linear compression" kernel on the
+ * page "Meta accelere un noyau GPU d'un facteur 4 avec TLX, une extension du langage
+ * Triton", sections "Comment le chargement des donnees gene le calcul" and "Ce que signifie
+ * une acceleration d'un facteur quatre": the operand common to every item (W) is read once
+ * per tile walk and never replicated per batch entry.
+ *
+ *   W      bf16, M x K row-major (shared by all b), ldw >= max(1, K).
+ *   X      bf16; X[b] = X + b*stride_x is K x N row-major ("N-major"), ldx >= max(1, N),
+ *          stride_x >= 0.
+ *   Y      out_type; Y[b] = Y + b*stride_y is M x N row-major, ldy >= max(1, N);
+ *          when batch > 1, stride_y >= (M-1)*ldy + N (output batches must not overlap).
+ * Same conventions and errors as gemm_bf16.  batch == 0: GEMM_OK, nothing enqueued.
+ */
+GEMM_API gemm_status_t gemm_bf16_batched_shared_w(int batch, int M, int N, int K, const void* W, int ldw,
+                                         const void* X, int ldx, long long stride_x, void* Y,
+                                         int ldy, long long stride_y, gemm_out_t out_type,
+                                         float alpha, float beta, struct CUstream_st* stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+GEMM_API const char* gemm_bf16_status_string(gemm_status_t s);
+
+/*
+ * gemm_bf16_device_status -- synchronizes `stream`, then reports whether any kernel of this
+ * library that ran on the current device since the previous call gave up a bounded
+ * barrier wait (GEMM_ERR_TIMEOUT; the word is then cleared), or GEMM_ERR_CUDA if the
+ * synchronization failed, else GEMM_OK.  A timed-out kernel skips its remaining tiles,
+ * releases its tensor memory and exits, so the CUDA context stays usable; its output is
+ * incomplete.
+ */
+GEMM_API gemm_status_t gemm_bf16_device_status(struct CUstream_st* stream);
+
+/*
+ * gemm_bf16_set_plan -- force a tile plan for all following calls in this process (for
+ * tuning sweeps and tests); -1 restores the automatic choice.
+ *   0: 128x128 tile, one CTA       1: 128x256 tile, one CTA
+ *   2: 256x256 tile, 2-CTA cluster 3: 256x128 tile, 2-CTA cluster
+ * Returns GEMM_ERR_INVALID_ARG for an unknown plan.  A plan that cannot serve a given
+ * call is replaced by the automatic choice for that call.
+ */
+GEMM_API gemm_status_t gemm_bf16_set_plan(int plan);
+
+/*
+ * gemm_bf16_set_wait_timeout_ns -- bound, in nanoseconds of the GPU global timer, of every
+ * barrier wait inside the kernels launched afterwards in this process (default 2e9 = 2 s;
+ * 0 restores the default).
+ */
+GEMM_API gemm_status_t gemm_bf16_set_wait_timeout_ns(unsigned long long ns);
+
+/* Library version as an integer (major*10000 + minor*100 + patch). */
+GEMM_API int gemm_bf16_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GEMM_BF16_H */

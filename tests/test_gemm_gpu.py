@@ -1,0 +1,297 @@
+"""GPU parity of the persistent tcgen05 GEMM against the fp64 oracle, through the C ABI.
+
+Every call goes through dsl_persistent_warp_b200 (ctypes -> libgemm_bf16.so).  Inputs are the
+seeded synthetic matrices of synth/; expected values come only from oracle/.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import bits_of, check, sample_rows, to_dev_bf16, values_f64
+from synth import bf16_bits_to_f64, f64_to_bf16_bits, matrix_bf16, seed_for
+
+pytestmark = pytest.mark.gpu
+
+PLANS = [0, 1, 2, 3]
+
+
+@pytest.fixture(scope="module")
+def pw():
+    import dsl_persistent_warp_b200 as m
+    yield m
+    m.capi.gemm_bf16_set_plan(-1)
+
+
+def _plan(pw, plan):
+    assert pw.capi.gemm_bf16_set_plan(plan) == 0
+
+
+def _run(pw, A, B, M, N, K, *, out=torch.bfloat16, alpha=1.0, beta=0.0, c0=None, ldc=None):
+    """A: (M, lda) uint16 bits, B: (N, ldb) bits.  Returns (C device tensor view, full buffer)."""
+    dA = to_dev_bf16(A)[:, :K]
+    dB = to_dev_bf16(B)[:, :K]
+    ldc = N if ldc is None else ldc
+    if c0 is None:
+        buf = torch.full((M, ldc), float("nan"), dtype=out, device="cuda")
+    else:
+        buf = c0.clone().cuda()
+    C = buf[:, :N]
+    pw.gemm_bf16(dA, dB, C, alpha=alpha, beta=beta)
+    torch.cuda.synchronize()
+    assert pw.device_status() == 0
+    return C, buf
+
+
+# ----------------------------------------------------------------------------- exactness
+@pytest.mark.parametrize("plan", PLANS)
+def test_integer_inputs_bit_exact(pw, plan):
+    """Small-integer inputs: every partial sum is an exact integer in fp32, so the GPU result
+    must equal the oracle bit for bit (fp32 out), and its single bf16 rounding (bf16 out)."""
+    _plan(pw, plan)
+    rng = np.random.default_rng(100 + plan)
+    M, N, K = 512, 384, 704
+    Ai = rng.integers(-2, 3, (M, K)).astype(np.float64)
+    Bi = rng.integers(-2, 3, (N, K)).astype(np.float64)
+    A, B = f64_to_bf16_bits(Ai), f64_to_bf16_bits(Bi)
+    Cref, _ = oracle.gemm(A, B, M=M, N=N, K=K)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.float32)
+    assert np.array_equal(values_f64(C), Cref)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16)
+    assert np.array_equal(bits_of(C), f64_to_bf16_bits(Cref))
+
+
+@pytest.mark.parametrize("plan", PLANS)
+def test_identity_and_permutation(pw, plan):
+    """A = I reproduces B^T exactly; a permutation permutes rows exactly."""
+    _plan(pw, plan)
+    n = 320
+    p = np.random.default_rng(7).permutation(n)
+    P = np.zeros((n, n))
+    P[np.arange(n), p] = 1.0
+    B = matrix_bf16(77, 200, n)
+    C, _ = _run(pw, f64_to_bf16_bits(P), B, n, 200, n, out=torch.float32)
+    assert np.array_equal(values_f64(C), bf16_bits_to_f64(B).T[p, :])
+
+
+# ----------------------------------------------------------------------------- config 1
+@pytest.mark.parametrize("plan", PLANS)
+def test_square_256_uniform_fp32(pw, plan):
+    """M=N=K=256, U[-1,1] inputs, fp32 output, alpha=1, beta=0."""
+    _plan(pw, plan)
+    M = N = K = 256
+    A = matrix_bf16(seed_for(0, "A"), M, K, dist="uniform")
+    B = matrix_bf16(seed_for(0, "B"), N, K, dist="uniform")
+    C, _ = _run(pw, A, B, M, N, K, out=torch.float32)
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K)
+    rep = check(values_f64(C), Cref, R, out_bf16=False)
+    assert rep["ok"], rep
+
+
+# ----------------------------------------------------------------------------- tails / edges
+TAIL_SHAPES = [(1, 1, 1), (1, 8, 1), (3, 5, 7), (129, 257, 65), (300, 200, 100), (127, 129, 1000),
+               (513, 264, 72), (64, 1000, 40), (1000, 16, 130)]
+
+
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("shape", TAIL_SHAPES, ids=[f"{m}x{n}x{k}" for m, n, k in TAIL_SHAPES])
+def test_ragged_shapes(pw, plan, shape):
+    """Tile tails in M, N and K (TMA zero fill, clipped stores), bf16 and fp32 outputs, with
+    alpha/beta and C read in place."""
+    _plan(pw, plan)
+    M, N, K = shape
+    A = matrix_bf16(11, M, K, ld=K + (8 - K % 8) % 8)
+    B = matrix_bf16(12, N, K, ld=K + (8 - K % 8) % 8)
+    for out in (torch.float32, torch.bfloat16):
+        ldc = N + (8 - N % 8) % 8 + 8
+        c0bits = matrix_bf16(13, M, N, ld=ldc)
+        c0 = torch.from_numpy(bf16_bits_to_f64(c0bits)).to(out)
+        C, buf = _run(pw, A, B, M, N, K, out=out, alpha=0.5, beta=1.0, c0=c0, ldc=ldc)
+        c0_np = c0[:, :N].to(torch.float32).numpy()
+        Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, c0=c0_np, alpha=0.5, beta=1.0)
+        rep = check(values_f64(C), Cref, R, out_bf16=out == torch.bfloat16)
+        assert rep["ok"], (out, rep)
+        # the ldc padding columns keep their canary values
+        pad_before = c0[:, N:].to(torch.float32).numpy()
+        pad_after = buf[:, N:].cpu().to(torch.float32).numpy()
+        assert np.array_equal(np.isnan(pad_before), np.isnan(pad_after))
+        assert np.array_equal(pad_before[~np.isnan(pad_before)], pad_after[~np.isnan(pad_after)])
+
+
+def test_beta_zero_ignores_nan_c(pw):
+    _plan(pw, -1)
+    M, N, K = 200, 136, 96
+    A = matrix_bf16(21, M, K)
+    B = matrix_bf16(22, N, K)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.float32)  # C starts as NaN
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K)
+    assert check(values_f64(C), Cref, R, out_bf16=False)["ok"]
+
+
+def test_k_zero_and_alpha_zero(pw):
+    _plan(pw, -1)
+    M, N = 70, 90
+    c0 = torch.randn(M, N, dtype=torch.float32)
+    C = c0.clone().cuda()
+    A = torch.empty((M, 0), dtype=torch.bfloat16, device="cuda")
+    B = torch.empty((N, 0), dtype=torch.bfloat16, device="cuda")
+    pw.gemm_bf16(A, B, C, alpha=1.0, beta=-2.0)
+    torch.cuda.synchronize()
+    assert torch.equal(C.cpu(), -2.0 * c0)
+    Ab = to_dev_bf16(matrix_bf16(1, M, 64))
+    Bb = to_dev_bf16(matrix_bf16(2, N, 64))
+    C = torch.full((M, N), float("nan"), device="cuda")
+    pw.gemm_bf16(Ab, Bb, C, alpha=0.0, beta=0.0)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(C).item() == 0
+
+
+def test_unaligned_leading_dimensions(pw):
+    """lda/ldb not a multiple of 8 (pre-pass copy) and ldc odd (direct-store epilogue)."""
+    _plan(pw, -1)
+    M, N, K = 261, 133, 203
+    A = matrix_bf16(31, M, K, ld=K)  # lda = 203: not TMA-able
+    B = matrix_bf16(32, N, K, ld=K + 2)
+    ldc = N  # 133: odd
+    c0bits = matrix_bf16(33, M, N, ld=ldc)
+    c0 = torch.from_numpy(bf16_bits_to_f64(c0bits)).to(torch.bfloat16)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16, alpha=0.5, beta=1.0, c0=c0, ldc=ldc)
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, c0=c0bits, alpha=0.5, beta=1.0)
+    rep = check(values_f64(C), Cref, R, out_bf16=True)
+    assert rep["ok"], rep
+
+
+def test_misaligned_base_pointer(pw):
+    """A base that is 2-byte but not 16-byte aligned goes through the pre-pass copy."""
+    _plan(pw, -1)
+    M, N, K = 150, 140, 128
+    Abits = matrix_bf16(41, M * K + 1, 1).reshape(-1)
+    Bbits = matrix_bf16(42, N, K)
+    dA_full = to_dev_bf16(Abits)
+    dA = dA_full[1:].view(M, K)
+    C = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    pw.gemm_bf16(dA, to_dev_bf16(Bbits), C)
+    torch.cuda.synchronize()
+    Cref, R = oracle.gemm(Abits[1:].reshape(M, K), Bbits, M=M, N=N, K=K)
+    assert check(values_f64(C), Cref, R, out_bf16=False)["ok"]
+
+
+@pytest.mark.parametrize("plan", PLANS)
+def test_deterministic(pw, plan):
+    _plan(pw, plan)
+    M, N, K = 700, 900, 1100
+    A = to_dev_bf16(matrix_bf16(51, M, K))
+    B = to_dev_bf16(matrix_bf16(52, N, K))
+    C1 = pw.gemm_bf16(A, B, out_dtype=torch.float32)
+    C2 = pw.gemm_bf16(A, B, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(C1, C2)
+
+
+def test_abi_errors_on_gpu(pw):
+    c = pw.capi
+    t = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    p = t.data_ptr()
+    s = torch.cuda.current_stream().cuda_stream
+    assert c.gemm_bf16(4, 4, 4, p, 3, p, 4, p, 4, 1, 1.0, 0.0, s) == c.GEMM_ERR_INVALID_ARG
+    assert c.gemm_bf16(4, 4, 4, p, 4, p, 4, p, 4, 7, 1.0, 0.0, s) == c.GEMM_ERR_INVALID_ARG
+    assert c.gemm_bf16(4, 4, 4, p + 1, 4, p, 4, p, 4, 1, 1.0, 0.0, s) == c.GEMM_ERR_INVALID_ARG
+    assert c.gemm_bf16(4, 4, 4, None, 4, p, 4, p, 4, 1, 1.0, 0.0, s) == c.GEMM_ERR_INVALID_ARG
+    assert c.gemm_bf16(4, 4, 4, p, 4, p, 4, p + 2, 4, 0, 1.0, 0.0, s) == c.GEMM_ERR_INVALID_ARG
+    assert c.gemm_bf16(0, 4, 4, None, 4, None, 4, None, 4, 1, 1.0, 0.0, s) == c.GEMM_OK
+    torch.cuda.synchronize()
+
+
+# ----------------------------------------------------------------------------- batched
+BATCH_CASES = [(3, 256, 128, 512), (5, 100, 72, 200), (2, 300, 264, 130), (64, 256, 128, 512)]
+
+
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("case", BATCH_CASES, ids=[f"b{b}_{m}x{n}x{k}" for b, m, n, k in BATCH_CASES])
+def test_batched_shared_w(pw, plan, case):
+    _plan(pw, plan)
+    batch, M, N, K = case
+    ldx = N + (8 - N % 8) % 8
+    W = matrix_bf16(61, M, K, std=512 ** -0.5)
+    X = matrix_bf16(62, batch * K, N, ld=ldx)
+    for out, beta in ((torch.bfloat16, 0.0), (torch.float32, 1.0)):
+        dW = to_dev_bf16(W)
+        dX = to_dev_bf16(X).view(batch, K, ldx)[:, :, :N]
+        y0 = torch.randn(batch, M, N, dtype=torch.float32).to(out)
+        Y = y0.clone().cuda()
+        pw.gemm_bf16_batched_shared_w(dW, dX, Y, alpha=1.0, beta=beta)
+        torch.cuda.synchronize()
+        assert pw.device_status() == 0
+        Cref, R = oracle.gemm_batched(W, X, batch=batch, M=M, N=N, K=K, stride_x=K * ldx,
+                                      y0=y0.to(torch.float32).numpy().reshape(batch * M, N),
+                                      stride_y=M * N, alpha=1.0, beta=beta)
+        rep = check(values_f64(Y), Cref, R, out_bf16=out == torch.bfloat16)
+        assert rep["ok"], (out, rep)
+
+
+# ----------------------------------------------------------------------------- full configs
+def _full_case(pw, idx, M, N, K, *, std_a=1.0, std_b=1.0, alpha=1.0, beta=0.0, rows=None):
+    _plan(pw, -1)
+    A = matrix_bf16(seed_for(idx, "A"), M, K, std=std_a)
+    B = matrix_bf16(seed_for(idx, "B"), N, K, std=std_b)
+    c0 = None
+    if beta != 0.0:
+        c0bits = matrix_bf16(seed_for(idx, "C"), M, N)
+        c0 = torch.from_numpy(c0bits.view(np.int16)).view(torch.bfloat16)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16, alpha=alpha, beta=beta, c0=c0)
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, c0=None if c0 is None else c0bits, alpha=alpha,
+                          beta=beta, rows=rows)
+    Cg = values_f64(C if rows is None else C[torch.as_tensor(rows, device="cuda")])
+    rep = check(Cg, Cref, R, out_bf16=True)
+    assert rep["ok"], rep
+    return C, A, B
+
+
+@pytest.mark.parametrize("n", [4096, 8192])
+def test_square_bf16(pw, n):
+    """M=N=K=4096 and 8192, N(0,1) inputs, bf16 output: sampled rows vs the oracle (every
+    output tile, both tile borders)."""
+    _full_case(pw, 1, n, n, n, rows=sample_rows(n, seed=n))
+
+
+@pytest.mark.parametrize("which", ["up", "down"])
+def test_llm_mlp_shapes(pw, which):
+    """LLM MLP GEMMs: up-proj 16384x28672x8192 and down-proj 16384x8192x28672, activations
+    N(0,1), weights N(0,0.02), bf16 out: sampled rows vs the oracle."""
+    M, N, K = (16384, 28672, 8192) if which == "up" else (16384, 8192, 28672)
+    _full_case(pw, 2, M, N, K, std_b=0.02, rows=sample_rows(M, seed=K, per_block=1))
+
+
+EDGE = [(4099, 4099, 4099), (8192, 256, 4096), (127, 8191, 2048)]
+
+
+@pytest.mark.parametrize("shape", EDGE, ids=[f"{m}x{n}x{k}" for m, n, k in EDGE])
+def test_edge_shapes(pw, shape):
+    """Edge shapes with alpha=0.5, beta=1 and C ~ N(0,1) bf16 in place (packed leading
+    dimensions, so 4099 and 8191 take the alignment pre-pass / direct-store paths)."""
+    M, N, K = shape
+    rows = None if M * N * K <= 8192 * 256 * 4096 else sample_rows(M, seed=M)
+    _full_case(pw, 3, M, N, K, alpha=0.5, beta=1.0, rows=rows)
+
+
+def test_recsys_batched_config(pw):
+    """Y[b] = W X[b], b < 2048, W 256x512 ~ N(0, 1/sqrt(512)), X[b] 512x128 ~ N(0,1), bf16 out.
+    All batches on sampled rows, and 16 whole batches."""
+    _plan(pw, -1)
+    batch, M, K, N = 2048, 256, 512, 128
+    W = matrix_bf16(seed_for(4, "W"), M, K, std=512 ** -0.5)
+    X = matrix_bf16(seed_for(4, "X"), batch * K, N)
+    dW, dX = to_dev_bf16(W), to_dev_bf16(X).view(batch, K, N)
+    Y = pw.gemm_bf16_batched_shared_w(dW, dX)
+    torch.cuda.synchronize()
+    assert pw.device_status() == 0
+    rows = [0, 1, 77, 127, 128, 200, 255]
+    Cref, R = oracle.gemm_batched(W, X, batch=batch, M=M, N=N, K=K, stride_x=K * N, rows=rows)
+    Yv = values_f64(Y[:, rows, :])
+    rep = check(Yv, Cref, R, out_bf16=True)
+    assert rep["ok"], rep
+    sel = np.random.default_rng(4).choice(batch, 16, replace=False)
+    for b in sel:
+        Cb, Rb = oracle.gemm(W, X[b * K:(b + 1) * K], M=M, N=N, K=K, b_kmajor=False)
+        rep = check(values_f64(Y[int(b)]), Cb, Rb, out_bf16=True)
+        assert rep["ok"], (int(b), rep)
