@@ -133,7 +133,7 @@ class ClockSampler(threading.Thread):
         self.reasons = set()
         self.max_mhz = None
         self.ok = False
-        self._stop = threading.Event()
+        self._halt = threading.Event()
         try:
             import pynvml
             import torch
@@ -151,7 +151,7 @@ class ClockSampler(threading.Thread):
         if not self.ok:
             return
         nv = self.nv
-        while not self._stop.is_set():
+        while not self._halt.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
                 mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
@@ -163,7 +163,7 @@ class ClockSampler(threading.Thread):
             time.sleep(self.period)
 
     def stop(self):
-        self._stop.set()
+        self._halt.set()
         self.join(timeout=2)
         if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
@@ -196,13 +196,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (every rank takes part; NCCL or gloo)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_tflops(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: the FLOPs of all ranks' timed steps over the slowest rank's time."""
+    return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
 
 
 def make_inputs(w, torch):
@@ -273,7 +280,7 @@ def run_ours(args, w, wname):
     if pw.device_status() != 0:
         raise RuntimeError("kernel reported a bounded-wait timeout in the timed region")
     total_ms = max_over_ranks(total_ms, world)
-    value = flops * args.steps * world / (total_ms * 1e-3) / 1e12
+    value = aggregate_tflops(flops, args.steps, world, total_ms)
     avg_launch_ms = statistics.mean(per_launch_ms)
 
     # end to end through the public API with host buffers: H2D of the inputs from pinned
@@ -300,7 +307,7 @@ def run_ours(args, w, wname):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     h2d = hA.numel() * 2 + hB.numel() * 2 + (hC0.numel() * hC0.element_size() if hC0 is not None else 0)
     d2h = hC.numel() * hC.element_size()
-    e2e_value = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = aggregate_tflops(flops, e2e_steps, world, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -405,24 +412,26 @@ def run_reference(args, w, wname):
     # bounded sample: at most ~`ref_seconds` of CPU work over warmup + steps.
     total_steps = args.steps + args.warmup
     per_step_s = max(0.02, args.ref_seconds / max(total_steps, 1))
-    A = matrix_bf16(seed_for(idx, "A" if batch == 1 else "W"), M, K, dist=dist, std=std_a)
+    # Rows of A are a prefix of its seeded stream, so only the rows a step can use are drawn.
+    a_rows = min(M, 1024)
+    A = matrix_bf16(seed_for(idx, "A" if batch == 1 else "W"), a_rows, K, dist=dist, std=std_a)
     if batch == 1:
         B = matrix_bf16(seed_for(idx, "B"), N, K, dist=dist, std=std_b)
     else:
         B = matrix_bf16(seed_for(idx, "X"), K, N, dist=dist, std=std_b)
-    c0 = matrix_bf16(seed_for(idx, "C"), M, N) if beta != 0.0 else None
+    c0 = matrix_bf16(seed_for(idx, "C"), a_rows, N) if beta != 0.0 else None
 
     def one(nrows):
         rows = list(range(nrows))
         if batch == 1:
-            oracle.gemm(A, B, M=M, N=N, K=K, c0=c0, alpha=alpha, beta=beta, rows=rows)
+            oracle.gemm(A, B, M=a_rows, N=N, K=K, c0=c0, alpha=alpha, beta=beta, rows=rows)
         else:
-            oracle.gemm(A, B, M=M, N=N, K=K, b_kmajor=False, rows=rows)
+            oracle.gemm(A, B, M=a_rows, N=N, K=K, b_kmajor=False, rows=rows)
 
     t0 = time.perf_counter()
     one(1)
     per_row = max(time.perf_counter() - t0, 1e-6)
-    nrows = int(max(1, min(M, per_step_s / per_row)))
+    nrows = int(max(1, min(a_rows, per_step_s / per_row)))
     for _ in range(args.warmup):
         one(nrows)
     t0 = time.perf_counter()

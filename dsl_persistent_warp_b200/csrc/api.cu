@@ -321,6 +321,9 @@ gemm_status_t run(Req r) {
         p.ldc = r.ldc;
         p.stride_c = r.stride_c;
         p.c_tma = c_tma ? 1 : 0;
+        // Whole chunks up to the last 16-byte-aligned column may use tensor stores; when the row
+        // end itself is aligned, the clipped last chunk may too.
+        p.n_store_tma = ((long long)r.N * es) % 16 == 0 ? (int)round_up(r.N, stg_cols) : r.N;
         p.c_read = r.beta != 0.0f ? 1 : 0;
         p.timeout_ns = g_timeout_ns.load();
         switch (plan) {

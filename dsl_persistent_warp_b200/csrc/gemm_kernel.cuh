@@ -58,6 +58,9 @@ struct KParams {
     long long ldc;           // elements
     long long stride_c;      // elements between batches of C
     int c_tma;               // 1: epilogue uses TMA stores (aligned C), 0: direct stores
+    int n_store_tma;         // columns [0, n_store_tma) may be TMA-stored; a chunk reaching past
+                             // it (a row end that is not 16-byte aligned) is stored directly,
+                             // because a tensor store writes whole 16-byte granules
     int c_read;              // 1: beta != 0
     unsigned long long timeout_ns;
 };
@@ -395,7 +398,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, STAGES, B_MN, OUT>::THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
                 }
-                if (p.c_tma) {
+                if (p.c_tma && colc + T::STG_COLS <= p.n_store_tma) {
                     const uint32_t sb = stg + buf * T::STG_BYTES;
                     if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();

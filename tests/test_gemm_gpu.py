@@ -27,19 +27,25 @@ def _plan(pw, plan):
     assert pw.capi.gemm_bf16_set_plan(plan) == 0
 
 
+GUARD_ROWS = 3
+
+
 def _run(pw, A, B, M, N, K, *, out=torch.bfloat16, alpha=1.0, beta=0.0, c0=None, ldc=None):
-    """A: (M, lda) uint16 bits, B: (N, ldb) bits.  Returns (C device tensor view, full buffer)."""
+    """A: (M, lda) uint16 bits, B: (N, ldb) bits.  C lives in a buffer with GUARD_ROWS extra NaN
+    rows after row M-1; returns (C device view, buffer rows 0..M-1); the guard rows are checked
+    to be untouched here."""
     dA = to_dev_bf16(A)[:, :K]
     dB = to_dev_bf16(B)[:, :K]
     ldc = N if ldc is None else ldc
-    if c0 is None:
-        buf = torch.full((M, ldc), float("nan"), dtype=out, device="cuda")
-    else:
-        buf = c0.clone().cuda()
+    full = torch.full((M + GUARD_ROWS, ldc), float("nan"), dtype=out, device="cuda")
+    if c0 is not None:
+        full[:M].copy_(c0.cuda())
+    buf = full[:M]
     C = buf[:, :N]
     pw.gemm_bf16(dA, dB, C, alpha=alpha, beta=beta)
     torch.cuda.synchronize()
     assert pw.device_status() == 0
+    assert torch.isnan(full[M:]).all().item(), "rows after C were written"
     return C, buf
 
 
