@@ -35,7 +35,11 @@ SIGNATURES = {
     "gemm_bf16_set_plan": (_I, [_I]),
     "gemm_bf16_set_wait_timeout_ns": (_I, [ctypes.c_ulonglong]),
     "gemm_bf16_version": (_I, []),
+    "gemm_bf16_noalloc": (_I, [_I, _I, _I, _P, _I, _P, _I, _P, _I, _I, _F, _F, _P]),
 }
+
+# Size of the fixed device scratch used by gemm_bf16_noalloc (GEMM_BF16_NOALLOC_SCRATCH_BYTES).
+GEMM_BF16_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class GemmError(RuntimeError):
@@ -91,3 +95,8 @@ def gemm_bf16_set_wait_timeout_ns(ns: int) -> int:
 
 def gemm_bf16_version() -> int:
     return LIB.gemm_bf16_version()
+
+
+def gemm_bf16_noalloc(M, N, K, A, lda, B, ldb, C, ldc, out_type, alpha, beta, stream) -> int:
+    """gemm_bf16 without any device allocation (fixed 32 MiB library scratch)."""
+    return LIB.gemm_bf16_noalloc(M, N, K, A, lda, B, ldb, C, ldc, out_type, alpha, beta, stream)

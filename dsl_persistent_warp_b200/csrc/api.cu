@@ -339,6 +339,139 @@ gemm_status_t run(Req r) {
 
 }  // namespace
 
+// ------------------------------------------------------------------ allocation-free variant
+// Scratch of gemm_bf16_noalloc: the padded copies of A and B written by the alignment pre-pass
+// and read by the GEMM kernel.  Every device that loads this library holds it until the process
+// exits.  In host code this name is only a host-side stand-in, never a device address: kernels
+// are given the address that noalloc_scratch() obtains once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GEMM_BF16_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_scratch_mu;
+std::array<void*, kMaxDevices> g_scratch_ptr{};
+
+// Device address of the scratch on device `dev`, which must be the current device.  The first
+// call per device asks the runtime for it; later calls reuse the cached value.
+gemm_status_t noalloc_scratch(int dev, void** out) {
+    if (dev < 0 || dev >= kMaxDevices) return GEMM_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return GEMM_ERR_CUDA;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return GEMM_OK;
+}
+
+// The gemm_bf16 path with the pre-pass copies placed in the static scratch.
+gemm_status_t run_noalloc(Req r) {
+    gemm_status_t v = validate(r);
+    if (v != GEMM_OK) return v;
+    if (r.batch == 0 || r.M == 0 || r.N == 0) return GEMM_OK;
+    if (r.batch == 1) {
+        r.stride_b = r.b_mn ? (long long)r.K * r.ldb : (long long)r.N * r.ldb;
+        r.stride_c = (long long)r.M * r.ldc;
+    }
+    if (r.K == 0 || r.alpha == 0.0f) return launch_scale(r);
+
+    const bool a_ok = aligned(r.A, 16) && (r.lda % 8) == 0;
+    const long long b_rows = r.b_mn ? r.K : r.N;
+    const long long b_cols = r.b_mn ? r.N : r.K;
+    const bool b_ok = aligned(r.B, 16) && (r.ldb % 8) == 0 &&
+                      (r.batch == 1 || ((r.stride_b % 8) == 0 && r.stride_b >= b_rows * r.ldb));
+    long long lda_p = r.lda, ldb_p = r.ldb, sb_p = r.stride_b;
+    long long ws_a = 0, ws_b = 0;
+    if (!a_ok) {
+        lda_p = round_up(r.K, 8);
+        ws_a = round_up((long long)r.M * lda_p * 2, 256);
+    }
+    if (!b_ok) {
+        ldb_p = round_up(b_cols, 8);
+        sb_p = b_rows * ldb_p;
+        ws_b = round_up(sb_p * 2 * r.batch, 256);
+    }
+    if (ws_a + ws_b > (long long)GEMM_BF16_NOALLOC_SCRATCH_BYTES) return GEMM_ERR_INVALID_ARG;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GEMM_ERR_CUDA;
+    DevInfo di;
+    if (!device_info(dev, di)) return GEMM_ERR_CUDA;
+    if (di.major != 10 || di.minor != 0) return GEMM_ERR_UNSUPPORTED;
+
+    const void* A = r.A;
+    const void* B = r.B;
+    if (ws_a + ws_b) {
+        void* ws = nullptr;
+        gemm_status_t s = noalloc_scratch(dev, &ws);
+        if (s != GEMM_OK) return s;
+        if (!a_ok) {
+            launch_pad(r.A, r.lda, 0, ws, lda_p, 0, 1, r.M, r.K, r.stream);
+            A = ws;
+        }
+        if (!b_ok) {
+            void* dst = static_cast<char*>(ws) + ws_a;
+            launch_pad(r.B, r.ldb, r.stride_b, dst, ldb_p, sb_p, r.batch, (int)b_rows, (int)b_cols,
+                       r.stream);
+            B = dst;
+        }
+    }
+
+    const int plan = choose_plan(r, di.sms);
+    const PlanDesc pd = kPlans[plan];
+    const int bn_cta = pd.bn / pd.cg;
+    const int es = r.out == OUT_F32 ? 4 : 2;
+    const int stg_cols = r.out == OUT_F32 ? 32 : 64;
+    const bool c_tma = aligned(r.C, 16) && ((r.ldc * es) % 16) == 0 &&
+                       (r.batch == 1 || ((r.stride_c * es) % 16) == 0);
+    CUtensorMap ma, mb, mc;
+    std::memset(&mc, 0, sizeof mc);
+    gemm_status_t st = encode_3d(&ma, A, false, (uint64_t)r.K, (uint64_t)r.M, 1, (uint64_t)lda_p * 2,
+                                 (uint64_t)lda_p * 2 * (uint64_t)r.M, 64, 128);
+    if (st == GEMM_OK) {
+        if (!r.b_mn)
+            st = encode_3d(&mb, B, false, (uint64_t)r.K, (uint64_t)r.N, (uint64_t)r.batch,
+                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, 64, (uint32_t)bn_cta);
+        else
+            st = encode_3d(&mb, B, false, (uint64_t)r.N, (uint64_t)r.K, (uint64_t)r.batch,
+                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, 64, 64);
+    }
+    if (st == GEMM_OK && c_tma)
+        st = encode_3d(&mc, r.C, r.out == OUT_F32, (uint64_t)r.N, (uint64_t)r.M, (uint64_t)r.batch,
+                       (uint64_t)r.ldc * es, (uint64_t)r.stride_c * es, (uint32_t)stg_cols, 32);
+    if (st != GEMM_OK) return st;
+    KParams p;
+    std::memset(&p, 0, sizeof p);
+    p.M = r.M;
+    p.N = r.N;
+    p.K = r.K;
+    p.m_blocks = (int)cdiv(r.M, 128 * pd.cg);
+    p.n_blocks = (int)cdiv(r.N, pd.bn);
+    p.batch = r.batch;
+    p.tiles = p.m_blocks * p.n_blocks * r.batch;
+    p.k_blocks = (int)cdiv(r.K, 64);
+    p.group_m = kGroupM;
+    p.alpha = r.alpha;
+    p.beta = r.beta;
+    p.C = r.C;
+    p.ldc = r.ldc;
+    p.stride_c = r.stride_c;
+    p.c_tma = c_tma ? 1 : 0;
+    p.n_store_tma = ((long long)r.N * es) % 16 == 0 ? (int)round_up(r.N, stg_cols) : r.N;
+    p.c_read = r.beta != 0.0f ? 1 : 0;
+    p.timeout_ns = g_timeout_ns.load();
+    switch (plan) {
+        case 0: return launch_plan<1, 128, 6>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
+        case 1: return launch_plan<1, 256, 4>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
+        case 2: return launch_plan<2, 256, 6>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
+        default: return launch_plan<2, 128, 8>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
+    }
+}
+
+}  // namespace
+
 extern "C" {
 
 gemm_status_t gemm_bf16(int M, int N, int K, const void* A, int lda, const void* B, int ldb, void* C,
@@ -359,6 +492,17 @@ gemm_status_t gemm_bf16_batched_shared_w(int batch, int M, int N, int K, const v
         Req r{batch, M, N, K, W, ldw, X, ldx, stride_x, true, Y, ldy, stride_y, (int)out_type,
               alpha, beta, stream};
         return run(r);
+    } catch (...) {
+        return GEMM_ERR_CUDA;
+    }
+}
+
+gemm_status_t gemm_bf16_noalloc(int M, int N, int K, const void* A, int lda, const void* B, int ldb,
+                                void* C, int ldc, gemm_out_t out_type, float alpha, float beta,
+                                cudaStream_t stream) {
+    try {
+        Req r{1, M, N, K, A, lda, B, ldb, 0, false, C, ldc, 0, (int)out_type, alpha, beta, stream};
+        return run_noalloc(r);
     } catch (...) {
         return GEMM_ERR_CUDA;
     }

@@ -125,6 +125,41 @@ GEMM_API gemm_status_t gemm_bf16_set_plan(int plan);
  */
 GEMM_API gemm_status_t gemm_bf16_set_wait_timeout_ns(unsigned long long ns);
 
+/*
+ * gemm_bf16_noalloc -- the same operation, arguments, layouts and errors as gemm_bf16, for
+ * callers that must not have this library allocate device memory.  (The pages describe no
+ * such entry point; it exists for integration only.)
+ *
+ * Who needs it: a caller whose device memory is already handed out by its own caching
+ * allocator or memory budget (a framework that reserves nearly all of the GPU, a service that
+ * pins a fixed footprint) cannot let a library draw extra memory from the device's pool, where
+ * the request may fail or fragment what the caller manages; a caller on a latency-critical
+ * path cannot afford the time an allocation may take.  gemm_bf16 may allocate a stream-ordered
+ * workspace when A or B is not laid out for the tensor-memory accelerator; this entry point
+ * never calls cudaMalloc, cudaMallocAsync, cudaFree or any allocating routine.
+ *
+ * Instead it uses one fixed scratch array of GEMM_BF16_NOALLOC_SCRATCH_BYTES (32 MiB) that
+ * lives in the library's device image: every GPU on which the library is used holds it until
+ * the process exits.  It stores the padded copies of A and/or B that the alignment pre-pass
+ * makes (needed when lda or ldb is not a multiple of 8 elements or a base is not 16-byte
+ * aligned).  If those copies, each rounded up to 256 bytes, need more than the scratch holds,
+ * the call returns GEMM_ERR_INVALID_ARG and enqueues nothing.  Calls whose operands need no
+ * copy do not touch the scratch.
+ *
+ * The scratch is shared by every call on a device and keeps the last call's contents; nothing
+ * in it has to start at zero (the copies are fully rewritten by each call that uses them, and
+ * their padding columns are never read).  Calls that use the scratch and overlap on the GPU
+ * (for instance on two streams without ordering between them) race on it: order them on one
+ * stream or with events.
+ *
+ * The first call on each device looks up the scratch's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it; make that first call before any stream capture.
+ */
+#define GEMM_BF16_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+GEMM_API gemm_status_t gemm_bf16_noalloc(int M, int N, int K, const void* A, int lda, const void* B,
+                                         int ldb, void* C, int ldc, gemm_out_t out_type,
+                                         float alpha, float beta, struct CUstream_st* stream);
+
 /* Library version as an integer (major*10000 + minor*100 + patch). */
 GEMM_API int gemm_bf16_version(void);
 
