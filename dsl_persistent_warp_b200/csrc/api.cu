@@ -86,11 +86,28 @@ struct Req {
 };
 
 struct PlanDesc {
-    int cg, bn, stages;
+    int cg, bn, nsub, stages;  // CTAs per tile, MMA N, N sub-tiles per tile, ring stages
 };
-constexpr PlanDesc kPlans[4] = {{1, 128, 6}, {1, 256, 4}, {2, 256, 6}, {2, 128, 8}};
+constexpr int kNumPlans = 5;
+constexpr PlanDesc kPlans[kNumPlans] = {
+    {1, 128, 1, 6},  // 0: 128x128, one CTA
+    {1, 256, 1, 4},  // 1: 128x256, one CTA
+    {2, 256, 1, 6},  // 2: 256x256, 2-CTA cluster
+    {2, 128, 1, 8},  // 3: 256x128, 2-CTA cluster
+    {2, 256, 2, 4},  // 4: 256x512, 2-CTA cluster, two 256-column MMA sub-tiles
+};
 
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+// m-blocks per raster group; GEMM_BF16_GROUP_M (1..64) overrides the default for tuning sweeps.
+int group_m() {
+    const char* e = std::getenv("GEMM_BF16_GROUP_M");
+    if (e) {
+        const int v = std::atoi(e);
+        if (v >= 1 && v <= 64) return v;
+    }
+    return kGroupM;
+}
 inline long long round_up(long long a, long long b) { return cdiv(a, b) * b; }
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -128,24 +145,37 @@ gemm_status_t encode_3d(CUtensorMap* m, const void* base, bool f32, uint64_t d0,
     return res == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_CUDA;
 }
 
+// Sustained rate of each plan with every SM busy (TFLOP/s measured on B200, 8192^3 bf16); only
+// the ratios matter.  The automatic choice minimises  waves * tile_flops / per-cluster rate:
+// large tiles move fewer operand bytes per FLOP, small tiles quantise better on small grids.
+constexpr double kPlanRate[kNumPlans] = {880.0, 1190.0, 1190.0, 790.0, 1400.0};
+
 // Plan for a request on a device with `sms` SMs (auto unless overridden).
 int choose_plan(const Req& r, int sms) {
     const int forced = g_plan_override.load();
     if (forced >= 0) return forced;
-    const long long t256x256 = cdiv(r.M, 256) * cdiv(r.N, 256) * r.batch;
-    const long long t256x128 = cdiv(r.M, 256) * cdiv(r.N, 128) * r.batch;
-    const long long t128x256 = cdiv(r.M, 128) * cdiv(r.N, 256) * r.batch;
-    if (t256x256 >= sms / 2) return 2;
-    if (t256x128 >= sms / 2) return 3;
-    if (t128x256 >= sms) return 1;
-    return 0;
+    int best = 0;
+    double best_t = 0.0;
+    for (int i = 0; i < kNumPlans; ++i) {
+        const PlanDesc& pd = kPlans[i];
+        const long long tm = 128LL * pd.cg, tn = (long long)pd.bn * pd.nsub;
+        const long long tiles = cdiv(r.M, tm) * cdiv(r.N, tn) * r.batch;
+        const long long slots = sms / pd.cg;
+        const long long waves = cdiv(tiles, slots);
+        const double t = (double)waves * (double)(tm * tn) * (double)slots / kPlanRate[i];
+        if (i == 0 || t < best_t * 0.999) {
+            best = i;
+            best_t = t;
+        }
+    }
+    return best;
 }
 
-template <int CG, int BN, int STAGES, int B_MN, int OUT>
+template <int CG, int BN, int NSUB, int STAGES, int B_MN, int OUT>
 gemm_status_t launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
                                 const KParams& p, int dev, int sms, cudaStream_t stream) {
-    using T = Tile<CG, BN, STAGES, B_MN, OUT>;
-    auto kern = gemm_persistent<CG, BN, STAGES, B_MN, OUT>;
+    using T = Tile<CG, BN, NSUB, STAGES, B_MN, OUT>;
+    auto kern = gemm_persistent<CG, BN, NSUB, STAGES, B_MN, OUT>;
     static std::array<std::atomic<int>, kMaxDevices> attr_done{};
     static std::array<std::atomic<int>, kMaxDevices> max_clusters{};
     if (!attr_done[dev].load()) {
@@ -190,19 +220,32 @@ gemm_status_t launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, co
     return cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, p) == cudaSuccess ? GEMM_OK : GEMM_ERR_CUDA;
 }
 
-template <int CG, int BN, int STAGES>
+template <int CG, int BN, int NSUB, int STAGES>
 gemm_status_t launch_plan(bool b_mn, int out, const CUtensorMap& ma, const CUtensorMap& mb,
                           const CUtensorMap& mc, const KParams& p, int dev, int sms, cudaStream_t st) {
     if (b_mn) {
         if constexpr ((BN / CG) % 64 == 0) {
-            return out == OUT_F32 ? launch_persistent<CG, BN, STAGES, 1, OUT_F32>(ma, mb, mc, p, dev, sms, st)
-                                  : launch_persistent<CG, BN, STAGES, 1, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
+            return out == OUT_F32
+                       ? launch_persistent<CG, BN, NSUB, STAGES, 1, OUT_F32>(ma, mb, mc, p, dev, sms, st)
+                       : launch_persistent<CG, BN, NSUB, STAGES, 1, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
         } else {
             return GEMM_ERR_UNSUPPORTED;
         }
     }
-    return out == OUT_F32 ? launch_persistent<CG, BN, STAGES, 0, OUT_F32>(ma, mb, mc, p, dev, sms, st)
-                          : launch_persistent<CG, BN, STAGES, 0, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
+    return out == OUT_F32 ? launch_persistent<CG, BN, NSUB, STAGES, 0, OUT_F32>(ma, mb, mc, p, dev, sms, st)
+                          : launch_persistent<CG, BN, NSUB, STAGES, 0, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
+}
+
+gemm_status_t launch_by_plan(int plan, bool b_mn, int out, const CUtensorMap& ma, const CUtensorMap& mb,
+                             const CUtensorMap& mc, const KParams& p, int dev, int sms, cudaStream_t st) {
+    switch (plan) {
+        case 0: return launch_plan<1, 128, 1, 6>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 1: return launch_plan<1, 256, 1, 4>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 2: return launch_plan<2, 256, 1, 6>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 3: return launch_plan<2, 128, 1, 8>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 4: return launch_plan<2, 256, 2, 4>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        default: return GEMM_ERR_INVALID_ARG;
+    }
 }
 
 gemm_status_t launch_scale(const Req& r) {
@@ -310,11 +353,11 @@ gemm_status_t run(Req r) {
         p.N = r.N;
         p.K = r.K;
         p.m_blocks = (int)cdiv(r.M, 128 * pd.cg);
-        p.n_blocks = (int)cdiv(r.N, pd.bn);
+        p.n_blocks = (int)cdiv(r.N, pd.bn * pd.nsub);
         p.batch = r.batch;
         p.tiles = p.m_blocks * p.n_blocks * r.batch;
         p.k_blocks = (int)cdiv(r.K, 64);
-        p.group_m = kGroupM;
+        p.group_m = group_m();
         p.alpha = r.alpha;
         p.beta = r.beta;
         p.C = r.C;
@@ -326,12 +369,7 @@ gemm_status_t run(Req r) {
         p.n_store_tma = ((long long)r.N * es) % 16 == 0 ? (int)round_up(r.N, stg_cols) : r.N;
         p.c_read = r.beta != 0.0f ? 1 : 0;
         p.timeout_ns = g_timeout_ns.load();
-        switch (plan) {
-            case 0: st = launch_plan<1, 128, 6>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream); break;
-            case 1: st = launch_plan<1, 256, 4>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream); break;
-            case 2: st = launch_plan<2, 256, 6>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream); break;
-            default: st = launch_plan<2, 128, 8>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream); break;
-        }
+        st = launch_by_plan(plan, r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
     }
     if (ws) cudaFreeAsync(ws, r.stream);
     return st;
@@ -448,11 +486,11 @@ gemm_status_t run_noalloc(Req r) {
     p.N = r.N;
     p.K = r.K;
     p.m_blocks = (int)cdiv(r.M, 128 * pd.cg);
-    p.n_blocks = (int)cdiv(r.N, pd.bn);
+    p.n_blocks = (int)cdiv(r.N, pd.bn * pd.nsub);
     p.batch = r.batch;
     p.tiles = p.m_blocks * p.n_blocks * r.batch;
     p.k_blocks = (int)cdiv(r.K, 64);
-    p.group_m = kGroupM;
+    p.group_m = group_m();
     p.alpha = r.alpha;
     p.beta = r.beta;
     p.C = r.C;
@@ -462,12 +500,7 @@ gemm_status_t run_noalloc(Req r) {
     p.n_store_tma = ((long long)r.N * es) % 16 == 0 ? (int)round_up(r.N, stg_cols) : r.N;
     p.c_read = r.beta != 0.0f ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
-    switch (plan) {
-        case 0: return launch_plan<1, 128, 6>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
-        case 1: return launch_plan<1, 256, 4>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
-        case 2: return launch_plan<2, 256, 6>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
-        default: return launch_plan<2, 128, 8>(r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
-    }
+    return launch_by_plan(plan, r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
 }
 
 }  // namespace
@@ -533,7 +566,7 @@ gemm_status_t gemm_bf16_device_status(cudaStream_t stream) {
 }
 
 gemm_status_t gemm_bf16_set_plan(int plan) {
-    if (plan < -1 || plan > 3) return GEMM_ERR_INVALID_ARG;
+    if (plan < -1 || plan >= kNumPlans) return GEMM_ERR_INVALID_ARG;
     g_plan_override.store(plan);
     return GEMM_OK;
 }

@@ -65,19 +65,27 @@ struct KParams {
     unsigned long long timeout_ns;
 };
 
-template <int CG, int BN, int STAGES, int B_MN, int OUT>
+// CG: CTAs per cluster tile (1, or 2 computing together with cta_group::2).  BN: N of one MMA,
+// i.e. the columns of one TMEM accumulator slot.  NSUB: MMA sub-tiles along N per tile (tile N =
+// BN * NSUB).  There are two accumulator slots: with NSUB == 1 they alternate between tiles (the
+// epilogue of a tile overlaps the next tile's mainloop); with NSUB == 2 a tile owns both, the
+// epilogue drains slot 0 while the last sub-tile 1 MMAs run, and the next tile starts in slot 0
+// as soon as it is drained.
+template <int CG, int BN, int NSUB, int STAGES, int B_MN, int OUT>
 struct Tile {
     static constexpr int BK = 64;                   // K per stage (128 B of bf16)
     static constexpr int BM = 128 * CG;             // rows of the cluster tile (MMA M)
-    static constexpr int BN_CTA = BN / CG;          // B rows (N) loaded by each CTA
+    static constexpr int TILE_N = BN * NSUB;        // columns of the cluster tile
+    static constexpr int BN_CTA = BN / CG;          // B rows (N) of one sub-tile loaded per CTA
     static constexpr int A_BYTES = 128 * BK * 2;
-    static constexpr int B_BYTES = BN_CTA * BK * 2;
+    static constexpr int B_SUB_BYTES = BN_CTA * BK * 2;
+    static constexpr int B_BYTES = NSUB * B_SUB_BYTES;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int EPI_WARPS = 4;
     static constexpr int THREADS = 32 * (2 + EPI_WARPS);
     static constexpr int STG_COLS = OUT == OUT_F32 ? 32 : 64;  // 128-byte rows
     static constexpr int STG_BYTES = 32 * 128;
-    static constexpr int CHUNKS = BN / STG_COLS;
+    static constexpr int CHUNKS = BN / STG_COLS;                // per accumulator slot
     static constexpr int TMEM_COLS = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128
                                    : 2 * BN <= 256 ? 256 : 512;
     static constexpr int OFF_A = 0;
@@ -89,6 +97,7 @@ struct Tile {
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
     static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack to align the base to 1 KiB
     static_assert(BN % (16 * CG) == 0 && BN <= 256, "MMA N");
+    static_assert(NSUB == 1 || NSUB == 2, "one or two sub-tiles");
     static_assert(!B_MN || BN_CTA % 64 == 0, "MN-major B is loaded in 64-column boxes");
     static_assert(BN % STG_COLS == 0, "epilogue chunks");
     static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
@@ -137,11 +146,11 @@ __device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint32_t 
     }
 }
 
-template <int CG, int BN, int STAGES, int B_MN, int OUT>
-__global__ void __launch_bounds__(Tile<CG, BN, STAGES, B_MN, OUT>::THREADS, 1)
+template <int CG, int BN, int NSUB, int STAGES, int B_MN, int OUT>
+__global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS, 1)
     gemm_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const KParams p) {
-    using T = Tile<CG, BN, STAGES, B_MN, OUT>;
+    using T = Tile<CG, BN, NSUB, STAGES, B_MN, OUT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -193,12 +202,11 @@ __global__ void __launch_bounds__(Tile<CG, BN, STAGES, B_MN, OUT>::THREADS, 1)
             const uint64_t pol = l2_policy_evict_normal();
             int stage = 0;
             uint32_t phase = 0;
-            for (int t = cluster_id; t < p.tiles; t += num_clusters) {
+            bool ok = true;
+            for (int t = cluster_id; ok && t < p.tiles; t += num_clusters) {
                 int b, mb, nb;
                 decode_tile(p, t, b, mb, nb);
                 const int a_row = mb * T::BM + (int)rank * 128;
-                const int b_row = nb * BN + (int)rank * T::BN_CTA;
-                bool ok = true;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!wait_phase<CG, false>(bar_empty(stage), phase ^ 1u, slot_abort, rank,
                                                p.timeout_ns, kStatusProducer)) {
@@ -207,28 +215,28 @@ __global__ void __launch_bounds__(Tile<CG, BN, STAGES, B_MN, OUT>::THREADS, 1)
                     }
                     const uint32_t full_local = bar_full(stage);
                     if (rank == 0) mbar_arrive_expect_tx(full_local, T::STAGE_BYTES * CG);
+                    const uint32_t full_bar = CG == 2 ? map_to_rank(full_local, 0) : full_local;
                     const uint32_t sa = sbase + T::OFF_A + stage * T::A_BYTES;
                     const uint32_t sb = sbase + T::OFF_B + stage * T::B_BYTES;
                     const int k0 = kb * T::BK;
-                    if constexpr (CG == 1) {
-                        tma_load_3d(sa, &tmA, full_local, k0, a_row, 0, pol);
+                    if constexpr (CG == 1) tma_load_3d(sa, &tmA, full_bar, k0, a_row, 0, pol);
+                    else tma_load_3d_pair(sa, &tmA, full_bar, k0, a_row, 0, pol);
+#pragma unroll
+                    for (int sub = 0; sub < NSUB; ++sub) {
+                        const int b_row = nb * T::TILE_N + sub * BN + (int)rank * T::BN_CTA;
+                        const uint32_t sbs = sb + sub * T::B_SUB_BYTES;
                         if constexpr (!B_MN) {
-                            tma_load_3d(sb, &tmB, full_local, k0, b_row, b, pol);
+                            if constexpr (CG == 1) tma_load_3d(sbs, &tmB, full_bar, k0, b_row, b, pol);
+                            else tma_load_3d_pair(sbs, &tmB, full_bar, k0, b_row, b, pol);
                         } else {
 #pragma unroll
-                            for (int j = 0; j < T::BN_CTA / 64; ++j)
-                                tma_load_3d(sb + j * 8192, &tmB, full_local, b_row + 64 * j, k0, b, pol);
-                        }
-                    } else {
-                        const uint32_t full_leader = map_to_rank(full_local, 0);
-                        tma_load_3d_pair(sa, &tmA, full_leader, k0, a_row, 0, pol);
-                        if constexpr (!B_MN) {
-                            tma_load_3d_pair(sb, &tmB, full_leader, k0, b_row, b, pol);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < T::BN_CTA / 64; ++j)
-                                tma_load_3d_pair(sb + j * 8192, &tmB, full_leader, b_row + 64 * j, k0, b,
-                                                 pol);
+                            for (int j = 0; j < T::BN_CTA / 64; ++j) {
+                                if constexpr (CG == 1)
+                                    tma_load_3d(sbs + j * 8192, &tmB, full_bar, b_row + 64 * j, k0, b, pol);
+                                else
+                                    tma_load_3d_pair(sbs + j * 8192, &tmB, full_bar, b_row + 64 * j, k0, b,
+                                                     pol);
+                            }
                         }
                     }
                     if (++stage == STAGES) {
@@ -236,7 +244,6 @@ __global__ void __launch_bounds__(Tile<CG, BN, STAGES, B_MN, OUT>::THREADS, 1)
                         phase ^= 1u;
                     }
                 }
-                if (!ok) break;
             }
         }
     } else if (warp == 1) {
@@ -245,15 +252,10 @@ __global__ void __launch_bounds__(Tile<CG, BN, STAGES, B_MN, OUT>::THREADS, 1)
             constexpr uint32_t IDESC = idesc_bf16_f32(T::BM, BN, 0, B_MN);
             int stage = 0;
             uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
-            for (int t = cluster_id; t < p.tiles; t += num_clusters) {
-                if (!wait_phase<CG, CG == 2>(bar_tempty(acc), acc_phase ^ 1u, slot_abort, rank,
-                                             p.timeout_ns, kStatusMma))
-                    break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                bool ok = true;
+            uint32_t tph[2] = {0u, 0u};  // phase bit of each accumulator slot's next use
+            int acc = 0;                 // slot of the tile when NSUB == 1
+            bool ok = true;
+            for (int t = cluster_id; ok && t < p.tiles; t += num_clusters) {
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, rank, p.timeout_ns,
                                                kStatusMma)) {
@@ -264,12 +266,37 @@ __global__ void __launch_bounds__(Tile<CG, BN, STAGES, B_MN, OUT>::THREADS, 1)
                     const uint32_t sa = sbase + T::OFF_A + stage * T::A_BYTES;
                     const uint32_t sb = sbase + T::OFF_B + stage * T::B_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < T::BK / 16; ++kk) {
-                        const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
-                        const uint64_t bdesc = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
-                                                    : smem_desc_sw128(sb + kk * 32, 16, 1024);
-                        umma_f16<CG>(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                    for (int sub = 0; sub < NSUB; ++sub) {
+                        const int slot = NSUB == 1 ? acc : sub;
+                        if (kb == 0) {
+                            // the slot must have been drained by the epilogue of its last use
+                            if (!wait_phase<CG, CG == 2>(bar_tempty(slot), tph[slot] ^ 1u, slot_abort, rank,
+                                                         p.timeout_ns, kStatusMma)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                        }
+                        const uint32_t d_tmem = tmem_base + (uint32_t)(slot * BN);
+                        const uint32_t sbs = sb + sub * T::B_SUB_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < T::BK / 16; ++kk) {
+                            const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
+                            const uint64_t bdesc = B_MN ? smem_desc_sw128(sbs + kk * 2048, 8192, 1024)
+                                                        : smem_desc_sw128(sbs + kk * 32, 16, 1024);
+                            umma_f16<CG>(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                        if (kb == p.k_blocks - 1) {
+                            // accumulator of this slot complete: hand it to the epilogue
+                            if constexpr (CG == 1) {
+                                umma_commit<1>(bar_tfull(slot));
+                            } else {
+                                umma_commit<2>(map_to_rank(bar_tfull(slot), 0));
+                                umma_commit<2>(map_to_rank(bar_tfull(slot), 1));
+                            }
+                        }
                     }
+                    if (!ok) break;
                     if constexpr (CG == 1) {
                         umma_commit<1>(bar_empty(stage));
                     } else {
@@ -281,15 +308,13 @@ __global__ void __launch_bounds__(Tile<CG, BN, STAGES, B_MN, OUT>::THREADS, 1)
                         phase ^= 1u;
                     }
                 }
-                if (!ok) break;
-                if constexpr (CG == 1) {
-                    umma_commit<1>(bar_tfull(acc));
+                if (NSUB == 1) {
+                    tph[acc] ^= 1u;
+                    acc ^= 1;
                 } else {
-                    umma_commit<2>(map_to_rank(bar_tfull(acc), 0));
-                    umma_commit<2>(map_to_rank(bar_tfull(acc), 1));
+                    tph[0] ^= 1u;
+                    tph[1] ^= 1u;
                 }
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1u;
             }
         }
     } else {
@@ -297,141 +322,148 @@ __global__ void __launch_bounds__(Tile<CG, BN, STAGES, B_MN, OUT>::THREADS, 1)
         const int ew = (int)warp - 2;       // 0..3
         const int q = (int)(warp & 3u);     // TMEM lane quarter this warp may access
         const uint32_t stg = sbase + T::OFF_STG + ew * 2 * T::STG_BYTES;
-        constexpr int ES = OUT == OUT_F32 ? 4 : 2;
         const uint32_t tempty_leader0 = CG == 2 ? map_to_rank(bar_tempty(0), 0) : bar_tempty(0);
+        uint32_t tph[2] = {0u, 0u};
         int acc = 0;
-        uint32_t acc_phase = 0;
         int buf = 0;
-        for (int t = cluster_id; t < p.tiles; t += num_clusters) {
+        bool ok = true;
+        for (int t = cluster_id; ok && t < p.tiles; t += num_clusters) {
             int b, mb, nb;
             decode_tile(p, t, b, mb, nb);
             const int row0 = mb * T::BM + (int)rank * 128 + 32 * q;
             const int row = row0 + (int)lane;
-            const int col0 = nb * BN;
-            int ok = 1;
-            if (lane == 0)
-                ok = wait_phase<CG, false>(bar_tfull(acc), acc_phase, slot_abort, rank, p.timeout_ns,
-                                           kStatusEpilogue);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
             const long long cbase = (long long)b * p.stride_c + (long long)row * p.ldc;
+            for (int sub = 0; sub < NSUB; ++sub) {
+                const int slot = NSUB == 1 ? acc : sub;
+                int w_ok = 1;
+                if (lane == 0)
+                    w_ok = wait_phase<CG, false>(bar_tfull(slot), tph[slot], slot_abort, rank, p.timeout_ns,
+                                                 kStatusEpilogue);
+                w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+                if (!w_ok) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                tph[slot] ^= 1u;
+                const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(slot * BN);
+                const int col0 = nb * T::TILE_N + sub * BN;
 #pragma unroll 1
-            for (int c = 0; c < T::CHUNKS; ++c) {
-                float v[T::STG_COLS];
-                {
-                    uint32_t r0[32];
-                    tmem_ld_32x32b_x32(trow + c * T::STG_COLS, r0);
-                    if constexpr (OUT == OUT_BF16) {
-                        uint32_t r1[32];
-                        tmem_ld_32x32b_x32(trow + c * T::STG_COLS + 32, r1);
-                        tmem_ld_wait(r0);
-                        tmem_ld_wait(r1);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[32 + j] = __uint_as_float(r1[j]);
-                    } else {
-                        tmem_ld_wait(r0);
-                    }
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
-                }
-                if (c == T::CHUNKS - 1) {
-                    // Accumulator drained: hand it back to the MMA warp (leader CTA).
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * acc);
-                }
-                const int colc = col0 + c * T::STG_COLS;
-                const bool row_in = row < p.M;
-                const bool full_cols = colc + T::STG_COLS <= p.N;
-#pragma unroll
-                for (int j = 0; j < T::STG_COLS; ++j) v[j] *= p.alpha;
-                if (p.c_read && row_in) {
-                    if (full_cols && p.c_tma) {
+                for (int c = 0; c < T::CHUNKS; ++c) {
+                    float v[T::STG_COLS];
+                    {
+                        uint32_t r0[32];
+                        tmem_ld_32x32b_x32(trow + c * T::STG_COLS, r0);
                         if constexpr (OUT == OUT_BF16) {
-                            const uint4* src = reinterpret_cast<const uint4*>(
-                                static_cast<const uint16_t*>(p.C) + cbase + colc);
+                            uint32_t r1[32];
+                            tmem_ld_32x32b_x32(trow + c * T::STG_COLS + 32, r1);
+                            tmem_ld_wait(r0);
+                            tmem_ld_wait(r1);
 #pragma unroll
-                            for (int j = 0; j < T::STG_COLS / 8; ++j) {
-                                const uint4 w = src[j];
-                                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                            for (int j = 0; j < 32; ++j) v[32 + j] = __uint_as_float(r1[j]);
+                        } else {
+                            tmem_ld_wait(r0);
+                        }
 #pragma unroll
-                                for (int h = 0; h < 4; ++h) {
-                                    v[8 * j + 2 * h] = fmaf(p.beta, __uint_as_float(ww[h] << 16), v[8 * j + 2 * h]);
-                                    v[8 * j + 2 * h + 1] =
-                                        fmaf(p.beta, __uint_as_float(ww[h] & 0xFFFF0000u), v[8 * j + 2 * h + 1]);
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
+                    }
+                    if (c == T::CHUNKS - 1) {
+                        // Slot drained: hand it back to the MMA warp (leader CTA).
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * slot);
+                    }
+                    const int colc = col0 + c * T::STG_COLS;
+                    const bool row_in = row < p.M;
+                    const bool full_cols = colc + T::STG_COLS <= p.N;
+#pragma unroll
+                    for (int j = 0; j < T::STG_COLS; ++j) v[j] *= p.alpha;
+                    if (p.c_read && row_in) {
+                        if (full_cols && p.c_tma) {
+                            if constexpr (OUT == OUT_BF16) {
+                                const uint4* src = reinterpret_cast<const uint4*>(
+                                    static_cast<const uint16_t*>(p.C) + cbase + colc);
+#pragma unroll
+                                for (int j = 0; j < T::STG_COLS / 8; ++j) {
+                                    const uint4 w = src[j];
+                                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                                    for (int h = 0; h < 4; ++h) {
+                                        v[8 * j + 2 * h] =
+                                            fmaf(p.beta, __uint_as_float(ww[h] << 16), v[8 * j + 2 * h]);
+                                        v[8 * j + 2 * h + 1] = fmaf(
+                                            p.beta, __uint_as_float(ww[h] & 0xFFFF0000u), v[8 * j + 2 * h + 1]);
+                                    }
+                                }
+                            } else {
+                                const float4* src = reinterpret_cast<const float4*>(
+                                    static_cast<const float*>(p.C) + cbase + colc);
+#pragma unroll
+                                for (int j = 0; j < T::STG_COLS / 4; ++j) {
+                                    const float4 w = src[j];
+                                    v[4 * j + 0] = fmaf(p.beta, w.x, v[4 * j + 0]);
+                                    v[4 * j + 1] = fmaf(p.beta, w.y, v[4 * j + 1]);
+                                    v[4 * j + 2] = fmaf(p.beta, w.z, v[4 * j + 2]);
+                                    v[4 * j + 3] = fmaf(p.beta, w.w, v[4 * j + 3]);
                                 }
                             }
                         } else {
-                            const float4* src = reinterpret_cast<const float4*>(
-                                static_cast<const float*>(p.C) + cbase + colc);
 #pragma unroll
-                            for (int j = 0; j < T::STG_COLS / 4; ++j) {
-                                const float4 w = src[j];
-                                v[4 * j + 0] = fmaf(p.beta, w.x, v[4 * j + 0]);
-                                v[4 * j + 1] = fmaf(p.beta, w.y, v[4 * j + 1]);
-                                v[4 * j + 2] = fmaf(p.beta, w.z, v[4 * j + 2]);
-                                v[4 * j + 3] = fmaf(p.beta, w.w, v[4 * j + 3]);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < T::STG_COLS; ++j) {
-                            if (colc + j < p.N) {
-                                float cin;
-                                if constexpr (OUT == OUT_BF16)
-                                    cin = __uint_as_float((uint32_t)(static_cast<const uint16_t*>(p.C)[cbase + colc + j]) << 16);
-                                else
-                                    cin = static_cast<const float*>(p.C)[cbase + colc + j];
-                                v[j] = fmaf(p.beta, cin, v[j]);
+                            for (int j = 0; j < T::STG_COLS; ++j) {
+                                if (colc + j < p.N) {
+                                    float cin;
+                                    if constexpr (OUT == OUT_BF16)
+                                        cin = __uint_as_float(
+                                            (uint32_t)(static_cast<const uint16_t*>(p.C)[cbase + colc + j]) << 16);
+                                    else
+                                        cin = static_cast<const float*>(p.C)[cbase + colc + j];
+                                    v[j] = fmaf(p.beta, cin, v[j]);
+                                }
                             }
                         }
                     }
-                }
-                // pack the 128-byte row segment into 8 x 16-byte words
-                uint32_t w[32];
-                if constexpr (OUT == OUT_BF16) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
-                }
-                if (p.c_tma && colc + T::STG_COLS <= p.n_store_tma) {
-                    const uint32_t sb = stg + buf * T::STG_BYTES;
-                    if (lane == 0) bulk_wait_group_read<1>();
-                    __syncwarp();
-                    const uint32_t row_addr = sb + lane * 128u;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        st_shared_v4(row_addr + ((uint32_t)(j ^ (int)(lane & 7u)) << 4), w[4 * j],
-                                     w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_3d(&tmC, sb, colc, row0, b);
-                        bulk_commit_group();
-                    }
-                    buf ^= 1;
-                } else if (row_in) {
+                    // pack the 128-byte row segment into 8 x 16-byte words
+                    uint32_t w[32];
                     if constexpr (OUT == OUT_BF16) {
-                        uint16_t* dst = static_cast<uint16_t*>(p.C) + cbase + colc;
 #pragma unroll
-                        for (int j = 0; j < T::STG_COLS; ++j)
-                            if (colc + j < p.N)
-                                dst[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
+                        for (int j = 0; j < 32; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
                     } else {
-                        float* dst = static_cast<float*>(p.C) + cbase + colc;
 #pragma unroll
-                        for (int j = 0; j < T::STG_COLS; ++j)
-                            if (colc + j < p.N) dst[j] = __uint_as_float(w[j]);
+                        for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
+                    }
+                    if (p.c_tma && colc + T::STG_COLS <= p.n_store_tma) {
+                        const uint32_t sbuf = stg + buf * T::STG_BYTES;
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                        const uint32_t row_addr = sbuf + lane * 128u;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            st_shared_v4(row_addr + ((uint32_t)(j ^ (int)(lane & 7u)) << 4), w[4 * j],
+                                         w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_3d(&tmC, sbuf, colc, row0, b);
+                            bulk_commit_group();
+                        }
+                        buf ^= 1;
+                    } else if (row_in) {
+                        if constexpr (OUT == OUT_BF16) {
+                            uint16_t* dst = static_cast<uint16_t*>(p.C) + cbase + colc;
+#pragma unroll
+                            for (int j = 0; j < T::STG_COLS; ++j)
+                                if (colc + j < p.N)
+                                    dst[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
+                        } else {
+                            float* dst = static_cast<float*>(p.C) + cbase + colc;
+#pragma unroll
+                            for (int j = 0; j < T::STG_COLS; ++j)
+                                if (colc + j < p.N) dst[j] = __uint_as_float(w[j]);
+                        }
                     }
                 }
-                (void)ES;
             }
-            acc ^= 1;
-            if (acc == 0) acc_phase ^= 1u;
+            if (NSUB == 1) acc ^= 1;
         }
         if (p.c_tma && lane == 0) bulk_wait_group_all();
     }

@@ -113,6 +113,7 @@ GEMM_API gemm_status_t gemm_bf16_device_status(struct CUstream_st* stream);
  * tuning sweeps and tests); -1 restores the automatic choice.
  *   0: 128x128 tile, one CTA       1: 128x256 tile, one CTA
  *   2: 256x256 tile, 2-CTA cluster 3: 256x128 tile, 2-CTA cluster
+ *   4: 256x512 tile, 2-CTA cluster (two 256-column MMA sub-tiles sharing the A tile)
  * Returns GEMM_ERR_INVALID_ARG for an unknown plan.  A plan that cannot serve a given
  * call is replaced by the automatic choice for that call.
  */

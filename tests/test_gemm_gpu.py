@@ -13,7 +13,7 @@ from synth import bf16_bits_to_f64, f64_to_bf16_bits, matrix_bf16, seed_for
 
 pytestmark = pytest.mark.gpu
 
-PLANS = [0, 1, 2, 3]
+PLANS = [0, 1, 2, 3, 4]
 
 
 @pytest.fixture(scope="module")
