@@ -86,15 +86,15 @@ struct Req {
 };
 
 struct PlanDesc {
-    int cg, bn, nsub, stages;  // CTAs per tile, MMA N, N sub-tiles per tile, ring stages
+    int cg, bn, nsub, stages, bk;  // CTAs per tile, MMA N, N sub-tiles per tile, ring stages, K per stage
 };
 constexpr int kNumPlans = 5;
 constexpr PlanDesc kPlans[kNumPlans] = {
-    {1, 128, 1, 6},  // 0: 128x128, one CTA
-    {1, 256, 1, 4},  // 1: 128x256, one CTA
-    {2, 256, 1, 6},  // 2: 256x256, 2-CTA cluster
-    {2, 128, 1, 8},  // 3: 256x128, 2-CTA cluster
-    {2, 256, 2, 4},  // 4: 256x512, 2-CTA cluster, two 256-column MMA sub-tiles
+    {1, 128, 1, 6, 64},  // 0: 128x128, one CTA
+    {1, 256, 1, 4, 64},  // 1: 128x256, one CTA
+    {2, 256, 1, 6, 64},  // 2: 256x256, 2-CTA cluster
+    {2, 128, 1, 8, 64},  // 3: 256x128, 2-CTA cluster
+    {2, 256, 2, 4, 64},  // 4: 256x512, 2-CTA cluster, two 256-column MMA sub-tiles
 };
 
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
@@ -131,7 +131,8 @@ gemm_status_t validate(const Req& r) {
 }
 
 gemm_status_t encode_3d(CUtensorMap* m, const void* base, bool f32, uint64_t d0, uint64_t d1,
-                        uint64_t d2, uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1) {
+                        uint64_t d2, uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1,
+                        CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return GEMM_ERR_CUDA;
     cuuint64_t dims[3] = {d0, d1, d2};
@@ -140,7 +141,7 @@ gemm_status_t encode_3d(CUtensorMap* m, const void* base, bool f32, uint64_t d0,
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult res = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                       const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return res == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_CUDA;
 }
@@ -171,11 +172,11 @@ int choose_plan(const Req& r, int sms) {
     return best;
 }
 
-template <int CG, int BN, int NSUB, int STAGES, int B_MN, int OUT>
+template <int CG, int BN, int NSUB, int STAGES, int BK, int B_MN, int OUT>
 gemm_status_t launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
                                 const KParams& p, int dev, int sms, cudaStream_t stream) {
-    using T = Tile<CG, BN, NSUB, STAGES, B_MN, OUT>;
-    auto kern = gemm_persistent<CG, BN, NSUB, STAGES, B_MN, OUT>;
+    using T = Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>;
+    auto kern = gemm_persistent<CG, BN, NSUB, STAGES, BK, B_MN, OUT>;
     static std::array<std::atomic<int>, kMaxDevices> attr_done{};
     static std::array<std::atomic<int>, kMaxDevices> max_clusters{};
     if (!attr_done[dev].load()) {
@@ -220,30 +221,30 @@ gemm_status_t launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, co
     return cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, p) == cudaSuccess ? GEMM_OK : GEMM_ERR_CUDA;
 }
 
-template <int CG, int BN, int NSUB, int STAGES>
+template <int CG, int BN, int NSUB, int STAGES, int BK>
 gemm_status_t launch_plan(bool b_mn, int out, const CUtensorMap& ma, const CUtensorMap& mb,
                           const CUtensorMap& mc, const KParams& p, int dev, int sms, cudaStream_t st) {
     if (b_mn) {
         if constexpr ((BN / CG) % 64 == 0) {
             return out == OUT_F32
-                       ? launch_persistent<CG, BN, NSUB, STAGES, 1, OUT_F32>(ma, mb, mc, p, dev, sms, st)
-                       : launch_persistent<CG, BN, NSUB, STAGES, 1, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
+                       ? launch_persistent<CG, BN, NSUB, STAGES, BK, 1, OUT_F32>(ma, mb, mc, p, dev, sms, st)
+                       : launch_persistent<CG, BN, NSUB, STAGES, BK, 1, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
         } else {
             return GEMM_ERR_UNSUPPORTED;
         }
     }
-    return out == OUT_F32 ? launch_persistent<CG, BN, NSUB, STAGES, 0, OUT_F32>(ma, mb, mc, p, dev, sms, st)
-                          : launch_persistent<CG, BN, NSUB, STAGES, 0, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
+    return out == OUT_F32 ? launch_persistent<CG, BN, NSUB, STAGES, BK, 0, OUT_F32>(ma, mb, mc, p, dev, sms, st)
+                          : launch_persistent<CG, BN, NSUB, STAGES, BK, 0, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
 }
 
 gemm_status_t launch_by_plan(int plan, bool b_mn, int out, const CUtensorMap& ma, const CUtensorMap& mb,
                              const CUtensorMap& mc, const KParams& p, int dev, int sms, cudaStream_t st) {
     switch (plan) {
-        case 0: return launch_plan<1, 128, 1, 6>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 1: return launch_plan<1, 256, 1, 4>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 2: return launch_plan<2, 256, 1, 6>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 3: return launch_plan<2, 128, 1, 8>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 4: return launch_plan<2, 256, 2, 4>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 0: return launch_plan<1, 128, 1, 6, 64>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 1: return launch_plan<1, 256, 1, 4, 64>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 2: return launch_plan<2, 256, 1, 6, 64>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 3: return launch_plan<2, 128, 1, 8, 64>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 4: return launch_plan<2, 256, 2, 4, 64>(b_mn, out, ma, mb, mc, p, dev, sms, st);
         default: return GEMM_ERR_INVALID_ARG;
     }
 }
@@ -325,7 +326,7 @@ gemm_status_t run(Req r) {
 
     const int plan = choose_plan(r, di.sms);
     const PlanDesc pd = kPlans[plan];
-    const int bn_cta = pd.bn / pd.cg;
+    const int b_chunk = pd.bn * pd.nsub / pd.cg;  // B rows per CTA and stage
     const int es = r.out == OUT_F32 ? 4 : 2;
     const int stg_cols = r.out == OUT_F32 ? 32 : 64;
     const bool c_tma = aligned(r.C, 16) && ((r.ldc * es) % 16) == 0 &&
@@ -333,15 +334,16 @@ gemm_status_t run(Req r) {
 
     CUtensorMap ma, mb, mc;
     std::memset(&mc, 0, sizeof mc);
+    const CUtensorMapSwizzle ksw = pd.bk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     gemm_status_t st = encode_3d(&ma, A, false, (uint64_t)r.K, (uint64_t)r.M, 1, (uint64_t)lda_p * 2,
-                                 (uint64_t)lda_p * 2 * (uint64_t)r.M, 64, 128);
+                                 (uint64_t)lda_p * 2 * (uint64_t)r.M, (uint32_t)pd.bk, 128, ksw);
     if (st == GEMM_OK) {
         if (!r.b_mn)
             st = encode_3d(&mb, B, false, (uint64_t)r.K, (uint64_t)r.N, (uint64_t)r.batch,
-                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, 64, (uint32_t)bn_cta);
+                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, (uint32_t)pd.bk, (uint32_t)b_chunk, ksw);
         else
             st = encode_3d(&mb, B, false, (uint64_t)r.N, (uint64_t)r.K, (uint64_t)r.batch,
-                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, 64, 64);
+                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, 64, (uint32_t)pd.bk);
     }
     if (st == GEMM_OK && c_tma)
         st = encode_3d(&mc, r.C, r.out == OUT_F32, (uint64_t)r.N, (uint64_t)r.M, (uint64_t)r.batch,
@@ -356,7 +358,7 @@ gemm_status_t run(Req r) {
         p.n_blocks = (int)cdiv(r.N, pd.bn * pd.nsub);
         p.batch = r.batch;
         p.tiles = p.m_blocks * p.n_blocks * r.batch;
-        p.k_blocks = (int)cdiv(r.K, 64);
+        p.k_blocks = (int)cdiv(r.K, pd.bk);
         p.group_m = group_m();
         p.alpha = r.alpha;
         p.beta = r.beta;
@@ -459,22 +461,23 @@ gemm_status_t run_noalloc(Req r) {
 
     const int plan = choose_plan(r, di.sms);
     const PlanDesc pd = kPlans[plan];
-    const int bn_cta = pd.bn / pd.cg;
+    const int b_chunk = pd.bn * pd.nsub / pd.cg;  // B rows per CTA and stage
     const int es = r.out == OUT_F32 ? 4 : 2;
     const int stg_cols = r.out == OUT_F32 ? 32 : 64;
     const bool c_tma = aligned(r.C, 16) && ((r.ldc * es) % 16) == 0 &&
                        (r.batch == 1 || ((r.stride_c * es) % 16) == 0);
     CUtensorMap ma, mb, mc;
     std::memset(&mc, 0, sizeof mc);
+    const CUtensorMapSwizzle ksw = pd.bk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     gemm_status_t st = encode_3d(&ma, A, false, (uint64_t)r.K, (uint64_t)r.M, 1, (uint64_t)lda_p * 2,
-                                 (uint64_t)lda_p * 2 * (uint64_t)r.M, 64, 128);
+                                 (uint64_t)lda_p * 2 * (uint64_t)r.M, (uint32_t)pd.bk, 128, ksw);
     if (st == GEMM_OK) {
         if (!r.b_mn)
             st = encode_3d(&mb, B, false, (uint64_t)r.K, (uint64_t)r.N, (uint64_t)r.batch,
-                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, 64, (uint32_t)bn_cta);
+                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, (uint32_t)pd.bk, (uint32_t)b_chunk, ksw);
         else
             st = encode_3d(&mb, B, false, (uint64_t)r.N, (uint64_t)r.K, (uint64_t)r.batch,
-                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, 64, 64);
+                           (uint64_t)ldb_p * 2, (uint64_t)sb_p * 2, 64, (uint32_t)pd.bk);
     }
     if (st == GEMM_OK && c_tma)
         st = encode_3d(&mc, r.C, r.out == OUT_F32, (uint64_t)r.N, (uint64_t)r.M, (uint64_t)r.batch,
@@ -489,7 +492,7 @@ gemm_status_t run_noalloc(Req r) {
     p.n_blocks = (int)cdiv(r.N, pd.bn * pd.nsub);
     p.batch = r.batch;
     p.tiles = p.m_blocks * p.n_blocks * r.batch;
-    p.k_blocks = (int)cdiv(r.K, 64);
+    p.k_blocks = (int)cdiv(r.K, pd.bk);
     p.group_m = group_m();
     p.alpha = r.alpha;
     p.beta = r.beta;

@@ -71,12 +71,13 @@ struct KParams {
 // epilogue of a tile overlaps the next tile's mainloop); with NSUB == 2 a tile owns both, the
 // epilogue drains slot 0 while the last sub-tile 1 MMAs run, and the next tile starts in slot 0
 // as soon as it is drained.
-template <int CG, int BN, int NSUB, int STAGES, int B_MN, int OUT>
+template <int CG, int BN, int NSUB, int STAGES, int BK_, int B_MN, int OUT>
 struct Tile {
-    static constexpr int BK = 64;                   // K per stage (128 B of bf16)
+    static constexpr int BK = BK_;                  // K per stage: 64 (128-B rows) or 32 (64-B rows)
     static constexpr int BM = 128 * CG;             // rows of the cluster tile (MMA M)
     static constexpr int TILE_N = BN * NSUB;        // columns of the cluster tile
-    static constexpr int BN_CTA = BN / CG;          // B rows (N) of one sub-tile loaded per CTA
+    static constexpr int BN_CTA = BN / CG;          // B rows (N) of one sub-tile held per CTA
+    static constexpr int B_CHUNK = NSUB * BN_CTA;   // contiguous B rows (tile columns) per CTA
     static constexpr int A_BYTES = 128 * BK * 2;
     static constexpr int B_SUB_BYTES = BN_CTA * BK * 2;
     static constexpr int B_BYTES = NSUB * B_SUB_BYTES;
@@ -99,7 +100,15 @@ struct Tile {
     static_assert(BN % (16 * CG) == 0 && BN <= 256, "MMA N");
     static_assert(NSUB == 1 || NSUB == 2, "one or two sub-tiles");
     static_assert(!B_MN || BN_CTA % 64 == 0, "MN-major B is loaded in 64-column boxes");
+    static_assert(B_CHUNK <= 256, "one tensor-map box per CTA and stage");
+    static_assert(BN_CTA % STG_COLS == 0, "an epilogue chunk maps to contiguous output columns");
     static_assert(BN % STG_COLS == 0, "epilogue chunks");
+    // K-major operands: one row of a stage is BK*2 bytes, swizzled at that width.
+    static constexpr uint32_t KMAJ_SWIZZLE = BK == 64 ? 2u : 4u;  // descriptor swizzle mode
+    static constexpr uint32_t KMAJ_SBO = 8u * BK * 2u;            // bytes between 8-row groups
+    // MN-major B: 64-column boxes of BK rows (128-byte rows, 128-byte swizzle).
+    static constexpr int MN_BOX_BYTES = 64 * 2 * BK;
+    static_assert(BK == 64 || BK == 32, "stage K");
     static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
 };
 
@@ -125,13 +134,11 @@ __device__ __forceinline__ void raise_abort(uint32_t slot_abort, uint32_t rank, 
     if constexpr (CG == 2) st_cluster_u32(map_to_rank(slot_abort, rank ^ 1u), 1u);
 }
 
-// Bounded wait on an mbarrier phase.  Returns false when the kernel is aborting (this wait
-// expired, or another role raised the abort flag).
+// Slow path of wait_phase: poll with the global-timer bound.
 template <int CG, bool CLUSTER_SCOPE>
-__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint32_t slot_abort,
-                                        uint32_t rank, unsigned long long timeout_ns,
-                                        unsigned int code) {
-    if (CLUSTER_SCOPE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, uint32_t slot_abort,
+                                             uint32_t rank, unsigned long long timeout_ns,
+                                             unsigned int code) {
     const uint64_t t0 = global_timer_ns();
     for (;;) {
 #pragma unroll 1
@@ -146,11 +153,22 @@ __device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint32_t 
     }
 }
 
-template <int CG, int BN, int NSUB, int STAGES, int B_MN, int OUT>
-__global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS, 1)
+// Bounded wait on an mbarrier phase.  Returns false when the kernel is aborting (this wait
+// expired, or another role raised the abort flag).  The first probe is inline: on the
+// critical path (a stage that is already full or free) it costs one instruction.
+template <int CG, bool CLUSTER_SCOPE>
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint32_t slot_abort,
+                                           uint32_t rank, unsigned long long timeout_ns,
+                                           unsigned int code) {
+    if (CLUSTER_SCOPE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    return wait_phase_slow<CG, CLUSTER_SCOPE>(bar, parity, slot_abort, rank, timeout_ns, code);
+}
+
+template <int CG, int BN, int NSUB, int STAGES, int BK, int B_MN, int OUT>
+__global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THREADS, 1)
     gemm_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const KParams p) {
-    using T = Tile<CG, BN, NSUB, STAGES, B_MN, OUT>;
+    using T = Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -199,7 +217,9 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint64_t pol = l2_policy_evict_normal();
+            const uint32_t full_leader0 = CG == 2 ? map_to_rank(bar_full(0), 0) : bar_full(0);
+            // A and B panels are read by several CTAs of a wave: keep them in L2.
+            const uint64_t pol = l2_policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -215,28 +235,25 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
                     }
                     const uint32_t full_local = bar_full(stage);
                     if (rank == 0) mbar_arrive_expect_tx(full_local, T::STAGE_BYTES * CG);
-                    const uint32_t full_bar = CG == 2 ? map_to_rank(full_local, 0) : full_local;
+                    const uint32_t full_bar = full_leader0 + 8u * stage;
                     const uint32_t sa = sbase + T::OFF_A + stage * T::A_BYTES;
                     const uint32_t sb = sbase + T::OFF_B + stage * T::B_BYTES;
                     const int k0 = kb * T::BK;
                     if constexpr (CG == 1) tma_load_3d(sa, &tmA, full_bar, k0, a_row, 0, pol);
                     else tma_load_3d_pair(sa, &tmA, full_bar, k0, a_row, 0, pol);
+                    // This CTA's B chunk: tile columns [rank*B_CHUNK, +B_CHUNK), contiguous.
+                    const int b_row = nb * T::TILE_N + (int)rank * T::B_CHUNK;
+                    if constexpr (!B_MN) {
+                        if constexpr (CG == 1) tma_load_3d(sb, &tmB, full_bar, k0, b_row, b, pol);
+                        else tma_load_3d_pair(sb, &tmB, full_bar, k0, b_row, b, pol);
+                    } else {
 #pragma unroll
-                    for (int sub = 0; sub < NSUB; ++sub) {
-                        const int b_row = nb * T::TILE_N + sub * BN + (int)rank * T::BN_CTA;
-                        const uint32_t sbs = sb + sub * T::B_SUB_BYTES;
-                        if constexpr (!B_MN) {
-                            if constexpr (CG == 1) tma_load_3d(sbs, &tmB, full_bar, k0, b_row, b, pol);
-                            else tma_load_3d_pair(sbs, &tmB, full_bar, k0, b_row, b, pol);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < T::BN_CTA / 64; ++j) {
-                                if constexpr (CG == 1)
-                                    tma_load_3d(sbs + j * 8192, &tmB, full_bar, b_row + 64 * j, k0, b, pol);
-                                else
-                                    tma_load_3d_pair(sbs + j * 8192, &tmB, full_bar, b_row + 64 * j, k0, b,
-                                                     pol);
-                            }
+                        for (int j = 0; j < T::B_CHUNK / 64; ++j) {
+                            if constexpr (CG == 1)
+                                tma_load_3d(sb + j * T::MN_BOX_BYTES, &tmB, full_bar, b_row + 64 * j, k0, b, pol);
+                            else
+                                tma_load_3d_pair(sb + j * T::MN_BOX_BYTES, &tmB, full_bar, b_row + 64 * j, k0, b,
+                                                 pol);
                         }
                     }
                     if (++stage == STAGES) {
@@ -250,9 +267,18 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && rank == 0) {
             constexpr uint32_t IDESC = idesc_bf16_f32(T::BM, BN, 0, B_MN);
+            // Descriptors of stage 0 (K step 0); other stages and K steps only add to the
+            // start-address field, which never carries out of its 14 bits (smem < 256 KiB).
+            const uint64_t adesc0 = smem_desc(sbase + T::OFF_A, 16, T::KMAJ_SBO, T::KMAJ_SWIZZLE);
+            const uint64_t bdesc0 = B_MN ? smem_desc(sbase + T::OFF_B, T::MN_BOX_BYTES, 1024, 2u)
+                                         : smem_desc(sbase + T::OFF_B, 16, T::KMAJ_SBO, T::KMAJ_SWIZZLE);
+            const uint32_t empty_r0 = CG == 2 ? map_to_rank(bar_empty(0), 0) : bar_empty(0);
+            const uint32_t empty_r1 = CG == 2 ? map_to_rank(bar_empty(0), 1) : bar_empty(0);
+            const uint32_t tfull_r0 = CG == 2 ? map_to_rank(bar_tfull(0), 0) : bar_tfull(0);
+            const uint32_t tfull_r1 = CG == 2 ? map_to_rank(bar_tfull(0), 1) : bar_tfull(0);
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t tph[2] = {0u, 0u};  // phase bit of each accumulator slot's next use
+            uint32_t tph = 0u;  // bit i: phase of accumulator slot i's next use
             int acc = 0;                 // slot of the tile when NSUB == 1
             bool ok = true;
             for (int t = cluster_id; ok && t < p.tiles; t += num_clusters) {
@@ -263,14 +289,15 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = sbase + T::OFF_A + stage * T::A_BYTES;
-                    const uint32_t sb = sbase + T::OFF_B + stage * T::B_BYTES;
+                    // descriptor start-address fields advance in 16-byte units
+                    const uint64_t a_st = adesc0 + (uint64_t)((stage * T::A_BYTES) >> 4);
+                    const uint64_t b_st = bdesc0 + (uint64_t)((stage * T::B_BYTES) >> 4);
 #pragma unroll
                     for (int sub = 0; sub < NSUB; ++sub) {
                         const int slot = NSUB == 1 ? acc : sub;
                         if (kb == 0) {
                             // the slot must have been drained by the epilogue of its last use
-                            if (!wait_phase<CG, CG == 2>(bar_tempty(slot), tph[slot] ^ 1u, slot_abort, rank,
+                            if (!wait_phase<CG, CG == 2>(bar_tempty(slot), ((tph >> slot) & 1u) ^ 1u, slot_abort, rank,
                                                          p.timeout_ns, kStatusMma)) {
                                 ok = false;
                                 break;
@@ -278,12 +305,12 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
                             tc_fence_after();
                         }
                         const uint32_t d_tmem = tmem_base + (uint32_t)(slot * BN);
-                        const uint32_t sbs = sb + sub * T::B_SUB_BYTES;
+                        const uint64_t b_sub = b_st + (uint64_t)((sub * T::B_SUB_BYTES) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < T::BK / 16; ++kk) {
-                            const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
-                            const uint64_t bdesc = B_MN ? smem_desc_sw128(sbs + kk * 2048, 8192, 1024)
-                                                        : smem_desc_sw128(sbs + kk * 32, 16, 1024);
+                            // K=16 step: 32 bytes along a K-major row; 16 rows (2 KiB) of an MN-major box
+                            const uint64_t adesc = a_st + (uint64_t)((kk * 32) >> 4);
+                            const uint64_t bdesc = b_sub + (uint64_t)((B_MN ? kk * 2048 : kk * 32) >> 4);
                             umma_f16<CG>(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
                         }
                         if (kb == p.k_blocks - 1) {
@@ -291,8 +318,8 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
                             if constexpr (CG == 1) {
                                 umma_commit<1>(bar_tfull(slot));
                             } else {
-                                umma_commit<2>(map_to_rank(bar_tfull(slot), 0));
-                                umma_commit<2>(map_to_rank(bar_tfull(slot), 1));
+                                umma_commit<2>(tfull_r0 + 8u * slot);
+                                umma_commit<2>(tfull_r1 + 8u * slot);
                             }
                         }
                     }
@@ -300,8 +327,8 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
                     if constexpr (CG == 1) {
                         umma_commit<1>(bar_empty(stage));
                     } else {
-                        umma_commit<2>(map_to_rank(bar_empty(stage), 0));
-                        umma_commit<2>(map_to_rank(bar_empty(stage), 1));
+                        umma_commit<2>(empty_r0 + 8u * stage);
+                        umma_commit<2>(empty_r1 + 8u * stage);
                     }
                     if (++stage == STAGES) {
                         stage = 0;
@@ -309,11 +336,10 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
                     }
                 }
                 if (NSUB == 1) {
-                    tph[acc] ^= 1u;
+                    tph ^= 1u << acc;
                     acc ^= 1;
                 } else {
-                    tph[0] ^= 1u;
-                    tph[1] ^= 1u;
+                    tph ^= 3u;
                 }
             }
         }
@@ -323,7 +349,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
         const int q = (int)(warp & 3u);     // TMEM lane quarter this warp may access
         const uint32_t stg = sbase + T::OFF_STG + ew * 2 * T::STG_BYTES;
         const uint32_t tempty_leader0 = CG == 2 ? map_to_rank(bar_tempty(0), 0) : bar_tempty(0);
-        uint32_t tph[2] = {0u, 0u};
+        uint32_t tph = 0u;
         int acc = 0;
         int buf = 0;
         bool ok = true;
@@ -337,7 +363,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
                 const int slot = NSUB == 1 ? acc : sub;
                 int w_ok = 1;
                 if (lane == 0)
-                    w_ok = wait_phase<CG, false>(bar_tfull(slot), tph[slot], slot_abort, rank, p.timeout_ns,
+                    w_ok = wait_phase<CG, false>(bar_tfull(slot), (tph >> slot) & 1u, slot_abort, rank, p.timeout_ns,
                                                  kStatusEpilogue);
                 w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
                 if (!w_ok) {
@@ -345,9 +371,11 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
                     break;
                 }
                 tc_fence_after();
-                tph[slot] ^= 1u;
+                tph ^= 1u << slot;
                 const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(slot * BN);
-                const int col0 = nb * T::TILE_N + sub * BN;
+                // MMA column j of sub-tile `sub` comes from CTA q = j / BN_CTA's B chunk, row
+                // sub*BN_CTA + j % BN_CTA of it, i.e. tile column q*B_CHUNK + sub*BN_CTA + j % BN_CTA.
+                const int col_tile = nb * T::TILE_N + sub * T::BN_CTA;
 #pragma unroll 1
                 for (int c = 0; c < T::CHUNKS; ++c) {
                     float v[T::STG_COLS];
@@ -373,7 +401,8 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, B_MN, OUT>::THREADS
                         __syncwarp();
                         if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * slot);
                     }
-                    const int colc = col0 + c * T::STG_COLS;
+                    const int jc = c * T::STG_COLS;
+                    const int colc = col_tile + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
                     const bool row_in = row < p.M;
                     const bool full_cols = colc + T::STG_COLS <= p.N;
 #pragma unroll
