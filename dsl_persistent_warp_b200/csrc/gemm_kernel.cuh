@@ -82,7 +82,12 @@ struct Tile {
     static constexpr int B_SUB_BYTES = BN_CTA * BK * 2;
     static constexpr int B_BYTES = NSUB * B_SUB_BYTES;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    // Epilogue: 4 warps, one per TMEM lane quarter, each with two 4 KiB staging buffers (the TMA
+    // store of one chunk overlaps the next chunk's TMEM load and conversion).  8 warps (two per
+    // quarter, one buffer each) also work but measured no faster on B200.
     static constexpr int EPI_WARPS = 4;
+    static constexpr int EPI_HALVES = EPI_WARPS / 4;          // warps sharing a lane quarter
+    static constexpr int STG_BUFS = 8 / EPI_WARPS;            // staging buffers per warp
     static constexpr int THREADS = 32 * (2 + EPI_WARPS);
     static constexpr int STG_COLS = OUT == OUT_F32 ? 32 : 64;  // 128-byte rows
     static constexpr int STG_BYTES = 32 * 128;
@@ -92,7 +97,7 @@ struct Tile {
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
-    static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * 2 * STG_BYTES;
+    static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_BUFS * STG_BYTES;
     static constexpr int NUM_BARS = 2 * STAGES + 4;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
@@ -102,7 +107,7 @@ struct Tile {
     static_assert(!B_MN || BN_CTA % 64 == 0, "MN-major B is loaded in 64-column boxes");
     static_assert(B_CHUNK <= 256, "one tensor-map box per CTA and stage");
     static_assert(BN_CTA % STG_COLS == 0, "an epilogue chunk maps to contiguous output columns");
-    static_assert(BN % STG_COLS == 0, "epilogue chunks");
+    static_assert(BN % (STG_COLS * EPI_HALVES) == 0, "epilogue chunks split evenly between warps");
     // K-major operands: one row of a stage is BK*2 bytes, swizzled at that width.
     static constexpr uint32_t KMAJ_SWIZZLE = BK == 64 ? 2u : 4u;  // descriptor swizzle mode
     static constexpr uint32_t KMAJ_SBO = 8u * BK * 2u;            // bytes between 8-row groups
@@ -345,9 +350,11 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int ew = (int)warp - 2;       // 0..3
-        const int q = (int)(warp & 3u);     // TMEM lane quarter this warp may access
-        const uint32_t stg = sbase + T::OFF_STG + ew * 2 * T::STG_BYTES;
+        const int ew = (int)warp - 2;                 // 0..EPI_WARPS-1
+        const int q = (int)(warp & 3u);               // TMEM lane quarter this warp may access
+        const int half = ew / 4;                      // which part of the slot's columns
+        constexpr int CPW = T::CHUNKS / T::EPI_HALVES;  // chunks per warp and slot
+        const uint32_t stg = sbase + T::OFF_STG + ew * T::STG_BUFS * T::STG_BYTES;
         const uint32_t tempty_leader0 = CG == 2 ? map_to_rank(bar_tempty(0), 0) : bar_tempty(0);
         uint32_t tph = 0u;
         int acc = 0;
@@ -377,7 +384,8 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
                 // sub*BN_CTA + j % BN_CTA of it, i.e. tile column q*B_CHUNK + sub*BN_CTA + j % BN_CTA.
                 const int col_tile = nb * T::TILE_N + sub * T::BN_CTA;
 #pragma unroll 1
-                for (int c = 0; c < T::CHUNKS; ++c) {
+                for (int ci = 0; ci < CPW; ++ci) {
+                    const int c = half * CPW + ci;
                     float v[T::STG_COLS];
                     {
                         uint32_t r0[32];
@@ -395,7 +403,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
                     }
-                    if (c == T::CHUNKS - 1) {
+                    if (ci == CPW - 1) {
                         // Slot drained: hand it back to the MMA warp (leader CTA).
                         tc_fence_before();
                         __syncwarp();
@@ -462,7 +470,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
                     }
                     if (p.c_tma && colc + T::STG_COLS <= p.n_store_tma) {
                         const uint32_t sbuf = stg + buf * T::STG_BYTES;
-                        if (lane == 0) bulk_wait_group_read<1>();
+                        if (lane == 0) bulk_wait_group_read<T::STG_BUFS - 1>();
                         __syncwarp();
                         const uint32_t row_addr = sbuf + lane * 128u;
 #pragma unroll
@@ -475,7 +483,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
                             tma_store_3d(&tmC, sbuf, colc, row0, b);
                             bulk_commit_group();
                         }
-                        buf ^= 1;
+                        if (T::STG_BUFS == 2) buf ^= 1;
                     } else if (row_in) {
                         if constexpr (OUT == OUT_BF16) {
                             uint16_t* dst = static_cast<uint16_t*>(p.C) + cbase + colc;
