@@ -87,15 +87,28 @@ struct Req {
 
 struct PlanDesc {
     int cg, bn, nsub, stages, bk;  // CTAs per tile, MMA N, N sub-tiles per tile, ring stages, K per stage
+    int ares;                      // A resident in shared memory (needs M <= 128*cg, K <= 512)
 };
-constexpr int kNumPlans = 5;
+constexpr int kNumPlans = 8;
+constexpr int kNumStreamPlans = 5;  // plans 0..4 stream both operands
 constexpr PlanDesc kPlans[kNumPlans] = {
-    {1, 128, 1, 6, 64},  // 0: 128x128, one CTA
-    {1, 256, 1, 4, 64},  // 1: 128x256, one CTA
-    {2, 256, 1, 6, 64},  // 2: 256x256, 2-CTA cluster
-    {2, 128, 1, 8, 64},  // 3: 256x128, 2-CTA cluster
-    {2, 256, 2, 4, 64},  // 4: 256x512, 2-CTA cluster, two 256-column MMA sub-tiles
+    {1, 128, 1, 6, 64, 0},  // 0: 128x128, one CTA
+    {1, 256, 1, 4, 64, 0},  // 1: 128x256, one CTA
+    {2, 256, 1, 6, 64, 0},  // 2: 256x256, 2-CTA cluster
+    {2, 128, 1, 8, 64, 0},  // 3: 256x128, 2-CTA cluster
+    {2, 256, 2, 4, 64, 0},  // 4: 256x512, 2-CTA cluster, two 256-column MMA sub-tiles
+    {2, 128, 1, 12, 64, 1},  // 5: 256x128, 2-CTA cluster, A resident (M <= 256, K <= 512)
+    {1, 128, 1, 6, 64, 1},   // 6: 128x128, one CTA, A resident (M <= 128, K <= 512)
+    {2, 256, 1, 6, 64, 1},   // 7: 256x256, 2-CTA cluster, A resident (M <= 256, K <= 512)
 };
+
+// Batch entries packed side by side into one tile by plan `pd` (1 = no packing): needs the
+// N-major (batched) B operand, N a multiple of the 64-column box and dividing the tile width.
+int pack_factor(const PlanDesc& pd, bool b_mn, int N) {
+    const int tile_n = pd.bn * pd.nsub;
+    if (!b_mn || N <= 0 || N % 64 != 0 || tile_n % N != 0 || tile_n == N) return 1;
+    return tile_n / N;
+}
 
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
@@ -149,18 +162,30 @@ gemm_status_t encode_3d(CUtensorMap* m, const void* base, bool f32, uint64_t d0,
 // Sustained rate of each plan with every SM busy (TFLOP/s measured on B200, 8192^3 bf16); only
 // the ratios matter.  The automatic choice minimises  waves * tile_flops / per-cluster rate:
 // large tiles move fewer operand bytes per FLOP, small tiles quantise better on small grids.
-constexpr double kPlanRate[kNumPlans] = {880.0, 1190.0, 1190.0, 790.0, 1400.0};
+constexpr double kPlanRate[kNumStreamPlans] = {880.0, 1190.0, 1190.0, 790.0, 1400.0};
+
+// Can plan `i` serve this request?
+bool plan_serves(int i, const Req& r) {
+    const PlanDesc& pd = kPlans[i];
+    if (pd.ares) return r.M <= 128 * pd.cg && r.K <= 8 * pd.bk;
+    return true;
+}
 
 // Plan for a request on a device with `sms` SMs (auto unless overridden).
 int choose_plan(const Req& r, int sms) {
     const int forced = g_plan_override.load();
-    if (forced >= 0) return forced;
+    if (forced >= 0 && plan_serves(forced, r)) return forced;
+    // Shared-W batched shapes with short K are bound by streaming X and Y through HBM: the
+    // 256x256 tile holding several batch entries side by side measured fastest (W re-reads hit
+    // L2); the resident-W plans (5-7) stay available through gemm_bf16_set_plan.
+    if (r.b_mn && r.K <= 1024 && pack_factor(kPlans[2], r.b_mn, r.N) > 1) return 2;
     int best = 0;
     double best_t = 0.0;
-    for (int i = 0; i < kNumPlans; ++i) {
+    for (int i = 0; i < kNumStreamPlans; ++i) {
         const PlanDesc& pd = kPlans[i];
         const long long tm = 128LL * pd.cg, tn = (long long)pd.bn * pd.nsub;
-        const long long tiles = cdiv(r.M, tm) * cdiv(r.N, tn) * r.batch;
+        const int pk = pack_factor(pd, r.b_mn, r.N);
+        const long long tiles = pk > 1 ? cdiv(r.M, tm) * cdiv(r.batch, pk) : cdiv(r.M, tm) * cdiv(r.N, tn) * r.batch;
         const long long slots = sms / pd.cg;
         const long long waves = cdiv(tiles, slots);
         const double t = (double)waves * (double)(tm * tn) * (double)slots / kPlanRate[i];
@@ -172,11 +197,11 @@ int choose_plan(const Req& r, int sms) {
     return best;
 }
 
-template <int CG, int BN, int NSUB, int STAGES, int BK, int B_MN, int OUT>
+template <int CG, int BN, int NSUB, int STAGES, int BK, int B_MN, int OUT, int ARES>
 gemm_status_t launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
                                 const KParams& p, int dev, int sms, cudaStream_t stream) {
-    using T = Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>;
-    auto kern = gemm_persistent<CG, BN, NSUB, STAGES, BK, B_MN, OUT>;
+    using T = Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES>;
+    auto kern = gemm_persistent<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES>;
     static std::array<std::atomic<int>, kMaxDevices> attr_done{};
     static std::array<std::atomic<int>, kMaxDevices> max_clusters{};
     if (!attr_done[dev].load()) {
@@ -221,30 +246,34 @@ gemm_status_t launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, co
     return cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, p) == cudaSuccess ? GEMM_OK : GEMM_ERR_CUDA;
 }
 
-template <int CG, int BN, int NSUB, int STAGES, int BK>
+template <int CG, int BN, int NSUB, int STAGES, int BK, int ARES>
 gemm_status_t launch_plan(bool b_mn, int out, const CUtensorMap& ma, const CUtensorMap& mb,
                           const CUtensorMap& mc, const KParams& p, int dev, int sms, cudaStream_t st) {
     if (b_mn) {
         if constexpr ((BN / CG) % 64 == 0) {
             return out == OUT_F32
-                       ? launch_persistent<CG, BN, NSUB, STAGES, BK, 1, OUT_F32>(ma, mb, mc, p, dev, sms, st)
-                       : launch_persistent<CG, BN, NSUB, STAGES, BK, 1, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
+                       ? launch_persistent<CG, BN, NSUB, STAGES, BK, 1, OUT_F32, ARES>(ma, mb, mc, p, dev, sms, st)
+                       : launch_persistent<CG, BN, NSUB, STAGES, BK, 1, OUT_BF16, ARES>(ma, mb, mc, p, dev, sms, st);
         } else {
             return GEMM_ERR_UNSUPPORTED;
         }
     }
-    return out == OUT_F32 ? launch_persistent<CG, BN, NSUB, STAGES, BK, 0, OUT_F32>(ma, mb, mc, p, dev, sms, st)
-                          : launch_persistent<CG, BN, NSUB, STAGES, BK, 0, OUT_BF16>(ma, mb, mc, p, dev, sms, st);
+    return out == OUT_F32
+               ? launch_persistent<CG, BN, NSUB, STAGES, BK, 0, OUT_F32, ARES>(ma, mb, mc, p, dev, sms, st)
+               : launch_persistent<CG, BN, NSUB, STAGES, BK, 0, OUT_BF16, ARES>(ma, mb, mc, p, dev, sms, st);
 }
 
 gemm_status_t launch_by_plan(int plan, bool b_mn, int out, const CUtensorMap& ma, const CUtensorMap& mb,
                              const CUtensorMap& mc, const KParams& p, int dev, int sms, cudaStream_t st) {
     switch (plan) {
-        case 0: return launch_plan<1, 128, 1, 6, 64>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 1: return launch_plan<1, 256, 1, 4, 64>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 2: return launch_plan<2, 256, 1, 6, 64>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 3: return launch_plan<2, 128, 1, 8, 64>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 4: return launch_plan<2, 256, 2, 4, 64>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 0: return launch_plan<1, 128, 1, 6, 64, 0>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 1: return launch_plan<1, 256, 1, 4, 64, 0>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 2: return launch_plan<2, 256, 1, 6, 64, 0>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 3: return launch_plan<2, 128, 1, 8, 64, 0>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 4: return launch_plan<2, 256, 2, 4, 64, 0>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 5: return launch_plan<2, 128, 1, 12, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 6: return launch_plan<1, 128, 1, 6, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 7: return launch_plan<2, 256, 1, 6, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
         default: return GEMM_ERR_INVALID_ARG;
     }
 }
@@ -355,9 +384,16 @@ gemm_status_t run(Req r) {
         p.N = r.N;
         p.K = r.K;
         p.m_blocks = (int)cdiv(r.M, 128 * pd.cg);
-        p.n_blocks = (int)cdiv(r.N, pd.bn * pd.nsub);
-        p.batch = r.batch;
-        p.tiles = p.m_blocks * p.n_blocks * r.batch;
+        p.pack = pack_factor(pd, r.b_mn, r.N);
+        p.batch_real = r.batch;
+        if (p.pack > 1) {
+            p.n_blocks = (int)cdiv(r.batch, p.pack);
+            p.batch = 1;
+        } else {
+            p.n_blocks = (int)cdiv(r.N, pd.bn * pd.nsub);
+            p.batch = r.batch;
+        }
+        p.tiles = p.m_blocks * p.n_blocks * p.batch;
         p.k_blocks = (int)cdiv(r.K, pd.bk);
         p.group_m = group_m();
         p.alpha = r.alpha;
@@ -489,9 +525,16 @@ gemm_status_t run_noalloc(Req r) {
     p.N = r.N;
     p.K = r.K;
     p.m_blocks = (int)cdiv(r.M, 128 * pd.cg);
-    p.n_blocks = (int)cdiv(r.N, pd.bn * pd.nsub);
-    p.batch = r.batch;
-    p.tiles = p.m_blocks * p.n_blocks * r.batch;
+    p.pack = pack_factor(pd, r.b_mn, r.N);
+    p.batch_real = r.batch;
+    if (p.pack > 1) {
+        p.n_blocks = (int)cdiv(r.batch, p.pack);
+        p.batch = 1;
+    } else {
+        p.n_blocks = (int)cdiv(r.N, pd.bn * pd.nsub);
+        p.batch = r.batch;
+    }
+    p.tiles = p.m_blocks * p.n_blocks * p.batch;
     p.k_blocks = (int)cdiv(r.K, pd.bk);
     p.group_m = group_m();
     p.alpha = r.alpha;

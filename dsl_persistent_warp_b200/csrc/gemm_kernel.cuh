@@ -62,6 +62,9 @@ struct KParams {
                              // it (a row end that is not 16-byte aligned) is stored directly,
                              // because a tensor store writes whole 16-byte granules
     int c_read;              // 1: beta != 0
+    int pack;                // batch entries side by side in one tile (MN-major B; 1 = none):
+                             // tile column c belongs to entry nb*pack + c/N, column c%N
+    int batch_real;          // number of batch entries (p.batch counts tile batches)
     unsigned long long timeout_ns;
 };
 
@@ -71,7 +74,10 @@ struct KParams {
 // epilogue of a tile overlaps the next tile's mainloop); with NSUB == 2 a tile owns both, the
 // epilogue drains slot 0 while the last sub-tile 1 MMAs run, and the next tile starts in slot 0
 // as soon as it is drained.
-template <int CG, int BN, int NSUB, int STAGES, int BK_, int B_MN, int OUT>
+// ARES: the A operand is resident -- the whole M x K panel of A (one M tile, K <= KB_RES * BK) is
+// loaded into shared memory once per CTA and the ring streams only B.  This is the shared-W
+// form: W is read from HBM once per CTA and never per batch entry.
+template <int CG, int BN, int NSUB, int STAGES, int BK_, int B_MN, int OUT, int ARES = 0>
 struct Tile {
     static constexpr int BK = BK_;                  // K per stage: 64 (128-B rows) or 32 (64-B rows)
     static constexpr int BM = 128 * CG;             // rows of the cluster tile (MMA M)
@@ -81,7 +87,8 @@ struct Tile {
     static constexpr int A_BYTES = 128 * BK * 2;
     static constexpr int B_SUB_BYTES = BN_CTA * BK * 2;
     static constexpr int B_BYTES = NSUB * B_SUB_BYTES;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int KB_RES = 8;                // resident k-blocks (K <= 512 at BK = 64)
+    static constexpr int STAGE_BYTES = (ARES ? 0 : A_BYTES) + B_BYTES;
     // Epilogue: 4 warps, one per TMEM lane quarter, each with two 4 KiB staging buffers (the TMA
     // store of one chunk overlaps the next chunk's TMEM load and conversion).  8 warps (two per
     // quarter, one buffer each) also work but measured no faster on B200.
@@ -95,10 +102,13 @@ struct Tile {
     static constexpr int TMEM_COLS = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128
                                    : 2 * BN <= 256 ? 256 : 512;
     static constexpr int OFF_A = 0;
-    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_B = OFF_A + (ARES ? KB_RES : STAGES) * A_BYTES;
     static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
-    static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_BUFS * STG_BYTES;
-    static constexpr int NUM_BARS = 2 * STAGES + 4;
+    // With A resident the epilogue stores rows straight from registers (no staging), leaving
+    // the shared memory to the B ring.
+    static constexpr int STG_REGION = ARES ? 0 : EPI_WARPS * STG_BUFS * STG_BYTES;
+    static constexpr int OFF_BAR = OFF_STG + STG_REGION;
+    static constexpr int NUM_BARS = 2 * STAGES + 5;  // full/empty ring, tfull/tempty slots, resident A
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16;
     static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack to align the base to 1 KiB
@@ -115,6 +125,7 @@ struct Tile {
     static constexpr int MN_BOX_BYTES = 64 * 2 * BK;
     static_assert(BK == 64 || BK == 32, "stage K");
     static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
+    static_assert(ARES == 0 || BK == 64, "resident A uses K=64 blocks");
 };
 
 // Tile t -> (batch, m-block, n-block); m-blocks are walked in groups of group_m so that
@@ -169,11 +180,11 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint32
     return wait_phase_slow<CG, CLUSTER_SCOPE>(bar, parity, slot_abort, rank, timeout_ns, code);
 }
 
-template <int CG, int BN, int NSUB, int STAGES, int BK, int B_MN, int OUT>
-__global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THREADS, 1)
+template <int CG, int BN, int NSUB, int STAGES, int BK, int B_MN, int OUT, int ARES>
+__global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES>::THREADS, 1)
     gemm_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const KParams p) {
-    using T = Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>;
+    using T = Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -190,6 +201,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
     auto bar_empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto bar_tfull = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
     auto bar_tempty = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+    const uint32_t bar_ares = bar0 + 8u * (2 * STAGES + 4);  // resident A landed
     const uint32_t slot_tmem = sbase + T::OFF_MISC;
     const uint32_t slot_abort = sbase + T::OFF_MISC + 4;
 
@@ -202,6 +214,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
             mbar_init(bar_tfull(a), 1);
             mbar_init(bar_tempty(a), T::EPI_WARPS * CG);
         }
+        mbar_init(bar_ares, 1);
         st_shared_volatile_u32(slot_abort, 0u);
         fence_mbarrier_init();
     }
@@ -228,6 +241,16 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            if constexpr (ARES != 0) {
+                // This CTA's 128 rows of the single M tile, every k-block, once.
+                if (rank == 0) mbar_arrive_expect_tx(bar_ares, (uint32_t)(T::A_BYTES * CG * p.k_blocks));
+                const uint32_t ares_bar = CG == 2 ? map_to_rank(bar_ares, 0) : bar_ares;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    const uint32_t sa = sbase + T::OFF_A + kb * T::A_BYTES;
+                    if constexpr (CG == 1) tma_load_3d(sa, &tmA, ares_bar, kb * T::BK, (int)rank * 128, 0, pol);
+                    else tma_load_3d_pair(sa, &tmA, ares_bar, kb * T::BK, (int)rank * 128, 0, pol);
+                }
+            }
             for (int t = cluster_id; ok && t < p.tiles; t += num_clusters) {
                 int b, mb, nb;
                 decode_tile(p, t, b, mb, nb);
@@ -244,8 +267,10 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
                     const uint32_t sa = sbase + T::OFF_A + stage * T::A_BYTES;
                     const uint32_t sb = sbase + T::OFF_B + stage * T::B_BYTES;
                     const int k0 = kb * T::BK;
-                    if constexpr (CG == 1) tma_load_3d(sa, &tmA, full_bar, k0, a_row, 0, pol);
-                    else tma_load_3d_pair(sa, &tmA, full_bar, k0, a_row, 0, pol);
+                    if constexpr (ARES == 0) {
+                        if constexpr (CG == 1) tma_load_3d(sa, &tmA, full_bar, k0, a_row, 0, pol);
+                        else tma_load_3d_pair(sa, &tmA, full_bar, k0, a_row, 0, pol);
+                    }
                     // This CTA's B chunk: tile columns [rank*B_CHUNK, +B_CHUNK), contiguous.
                     const int b_row = nb * T::TILE_N + (int)rank * T::B_CHUNK;
                     if constexpr (!B_MN) {
@@ -254,11 +279,14 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
                     } else {
 #pragma unroll
                         for (int j = 0; j < T::B_CHUNK / 64; ++j) {
+                            // 64-column box j; with packing it lies inside one batch entry (N % 64 == 0)
+                            const int tc = (int)rank * T::B_CHUNK + 64 * j;
+                            const int bx = p.pack > 1 ? nb * p.pack + tc / p.N : b;
+                            const int cx = p.pack > 1 ? tc % p.N : b_row + 64 * j;
                             if constexpr (CG == 1)
-                                tma_load_3d(sb + j * T::MN_BOX_BYTES, &tmB, full_bar, b_row + 64 * j, k0, b, pol);
+                                tma_load_3d(sb + j * T::MN_BOX_BYTES, &tmB, full_bar, cx, k0, bx, pol);
                             else
-                                tma_load_3d_pair(sb + j * T::MN_BOX_BYTES, &tmB, full_bar, b_row + 64 * j, k0, b,
-                                                 pol);
+                                tma_load_3d_pair(sb + j * T::MN_BOX_BYTES, &tmB, full_bar, cx, k0, bx, pol);
                         }
                     }
                     if (++stage == STAGES) {
@@ -286,6 +314,10 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
             uint32_t tph = 0u;  // bit i: phase of accumulator slot i's next use
             int acc = 0;                 // slot of the tile when NSUB == 1
             bool ok = true;
+            if constexpr (ARES != 0) {
+                ok = wait_phase<CG, false>(bar_ares, 0u, slot_abort, rank, p.timeout_ns, kStatusMma);
+                tc_fence_after();
+            }
             for (int t = cluster_id; ok && t < p.tiles; t += num_clusters) {
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, rank, p.timeout_ns,
@@ -295,7 +327,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
                     }
                     tc_fence_after();
                     // descriptor start-address fields advance in 16-byte units
-                    const uint64_t a_st = adesc0 + (uint64_t)((stage * T::A_BYTES) >> 4);
+                    const uint64_t a_st = adesc0 + (uint64_t)(((ARES ? kb : stage) * T::A_BYTES) >> 4);
                     const uint64_t b_st = bdesc0 + (uint64_t)((stage * T::B_BYTES) >> 4);
 #pragma unroll
                     for (int sub = 0; sub < NSUB; ++sub) {
@@ -365,7 +397,6 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
             decode_tile(p, t, b, mb, nb);
             const int row0 = mb * T::BM + (int)rank * 128 + 32 * q;
             const int row = row0 + (int)lane;
-            const long long cbase = (long long)b * p.stride_c + (long long)row * p.ldc;
             for (int sub = 0; sub < NSUB; ++sub) {
                 const int slot = NSUB == 1 ? acc : sub;
                 int w_ok = 1;
@@ -382,7 +413,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
                 const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(slot * BN);
                 // MMA column j of sub-tile `sub` comes from CTA q = j / BN_CTA's B chunk, row
                 // sub*BN_CTA + j % BN_CTA of it, i.e. tile column q*B_CHUNK + sub*BN_CTA + j % BN_CTA.
-                const int col_tile = nb * T::TILE_N + sub * T::BN_CTA;
+                const int col_tile = sub * T::BN_CTA;  // column within the tile
 #pragma unroll 1
                 for (int ci = 0; ci < CPW; ++ci) {
                     const int c = half * CPW + ci;
@@ -410,8 +441,11 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
                         if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * slot);
                     }
                     const int jc = c * T::STG_COLS;
-                    const int colc = col_tile + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
-                    const bool row_in = row < p.M;
+                    const int tcol = col_tile + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
+                    const int bb = p.pack > 1 ? nb * p.pack + tcol / p.N : b;
+                    const int colc = p.pack > 1 ? tcol % p.N : nb * T::TILE_N + tcol;
+                    const long long cbase = (long long)bb * p.stride_c + (long long)row * p.ldc;
+                    const bool row_in = row < p.M && bb < p.batch_real;
                     const bool full_cols = colc + T::STG_COLS <= p.N;
 #pragma unroll
                     for (int j = 0; j < T::STG_COLS; ++j) v[j] *= p.alpha;
@@ -468,7 +502,14 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
 #pragma unroll
                         for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
                     }
-                    if (p.c_tma && colc + T::STG_COLS <= p.n_store_tma) {
+                    if (ARES != 0 && p.c_tma && full_cols && row_in) {
+                        // whole 128-byte row segment of this thread, inside N: eight 16-byte stores
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<char*>(p.C) +
+                                                              (cbase + colc) * (OUT == OUT_BF16 ? 2 : 4));
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                    } else if (ARES == 0 && p.c_tma && colc + T::STG_COLS <= p.n_store_tma && bb < p.batch_real) {
                         const uint32_t sbuf = stg + buf * T::STG_BYTES;
                         if (lane == 0) bulk_wait_group_read<T::STG_BUFS - 1>();
                         __syncwarp();
@@ -480,7 +521,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT>::THR
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_3d(&tmC, sbuf, colc, row0, b);
+                            tma_store_3d(&tmC, sbuf, colc, row0, bb);
                             bulk_commit_group();
                         }
                         if (T::STG_BUFS == 2) buf ^= 1;

@@ -114,6 +114,11 @@ GEMM_API gemm_status_t gemm_bf16_device_status(struct CUstream_st* stream);
  *   0: 128x128 tile, one CTA       1: 128x256 tile, one CTA
  *   2: 256x256 tile, 2-CTA cluster 3: 256x128 tile, 2-CTA cluster
  *   4: 256x512 tile, 2-CTA cluster (two 256-column MMA sub-tiles sharing the A tile)
+ *   5: 256x128 tile, 2-CTA cluster, A resident in shared memory (M <= 256, K <= 512)
+ *   6: 128x128 tile, one CTA, A resident in shared memory (M <= 128, K <= 512)
+ *   7: 256x256 tile, 2-CTA cluster, A resident in shared memory (M <= 256, K <= 512)
+ * In the batched call, a tile wider than N holds several batch entries side by side when N is a
+ * multiple of 64 that divides the tile width.
  * Returns GEMM_ERR_INVALID_ARG for an unknown plan.  A plan that cannot serve a given
  * call is replaced by the automatic choice for that call.
  */

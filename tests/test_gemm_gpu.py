@@ -13,7 +13,7 @@ from synth import bf16_bits_to_f64, f64_to_bf16_bits, matrix_bf16, seed_for
 
 pytestmark = pytest.mark.gpu
 
-PLANS = [0, 1, 2, 3, 4]
+PLANS = [0, 1, 2, 3, 4, 5, 6, 7]
 
 
 @pytest.fixture(scope="module")
@@ -209,7 +209,10 @@ def test_abi_errors_on_gpu(pw):
 
 
 # ----------------------------------------------------------------------------- batched
-BATCH_CASES = [(3, 256, 128, 512), (5, 100, 72, 200), (2, 300, 264, 130), (64, 256, 128, 512)]
+# (batch, M, N, K).  N = 64, 128 or 256 lets wide tiles hold several batch entries side by side
+# (with an odd batch count the last tile is partly empty); N = 72 and 264 cannot be packed.
+BATCH_CASES = [(3, 256, 128, 512), (5, 100, 72, 200), (2, 300, 264, 130), (64, 256, 128, 512),
+               (5, 256, 64, 256), (7, 128, 128, 512), (3, 200, 256, 320)]
 
 
 @pytest.mark.parametrize("plan", PLANS)
