@@ -162,7 +162,7 @@ gemm_status_t encode_3d(CUtensorMap* m, const void* base, bool f32, uint64_t d0,
 // Sustained rate of each plan with every SM busy (TFLOP/s measured on B200, 8192^3 bf16); only
 // the ratios matter.  The automatic choice minimises  waves * tile_flops / per-cluster rate:
 // large tiles move fewer operand bytes per FLOP, small tiles quantise better on small grids.
-constexpr double kPlanRate[kNumStreamPlans] = {880.0, 1190.0, 1190.0, 790.0, 1400.0};
+constexpr double kPlanRate[kNumStreamPlans] = {880.0, 1190.0, 1250.0, 790.0, 1400.0};
 
 // Can plan `i` serve this request?
 bool plan_serves(int i, const Req& r) {
@@ -299,9 +299,12 @@ void launch_pad(const void* src, long long ld_src, long long bs_src, void* dst, 
     if (gx > 8) gx = 8;
     int gy = rows < 4096 ? (rows > 0 ? rows : 1) : 4096;
     int gz = batch < 65535 ? batch : 65535;
+    // extent of the source: from its first element to one past its last
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(src);
+    const uintptr_t hi = lo + 2 * (uintptr_t)((long long)(batch - 1) * bs_src + (long long)(rows - 1) * ld_src + cols);
     pad_copy_kernel<<<dim3(gx, gy, gz), threads, 0, st>>>(
         static_cast<const uint16_t*>(src), ld_src, bs_src, static_cast<uint16_t*>(dst), ld_dst, bs_dst,
-        batch, rows, cols);
+        batch, rows, cols, lo, hi);
 }
 
 gemm_status_t run(Req r) {

@@ -447,9 +447,85 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     const long long cbase = (long long)bb * p.stride_c + (long long)row * p.ldc;
                     const bool row_in = row < p.M && bb < p.batch_real;
                     const bool full_cols = colc + T::STG_COLS <= p.N;
+                    // A chunk goes out as one tensor store when C is TMA-addressable up to the
+                    // chunk's end; otherwise (unaligned ldc, a ragged right edge) the warp moves it
+                    // row by row through the staging buffer so that every access is coalesced.
+                    const bool tma_chunk =
+                        ARES == 0 && p.c_tma && colc + T::STG_COLS <= p.n_store_tma && bb < p.batch_real;
+                    const bool coop_chunk = ARES == 0 && !tma_chunk;
+                    const uint32_t sbuf = stg + buf * T::STG_BYTES;
+                    if (ARES == 0) {
+                        // the buffer may still be read by an earlier tensor store
+                        if (lane == 0) bulk_wait_group_read<T::STG_BUFS - 1>();
+                        __syncwarp();
+                    }
 #pragma unroll
                     for (int j = 0; j < T::STG_COLS; ++j) v[j] *= p.alpha;
-                    if (p.c_read && row_in) {
+                    if (p.c_read && coop_chunk) {
+                        // C_in: lane j reads elements j (and j+32 for bf16) of each of the warp's 32
+                        // rows; element e of row r sits in 16-byte chunk (e*ES/16) ^ (r & 7).  Rows
+                        // go 8 at a time so that 8 (16 for bf16) loads per lane are in flight.
+                        constexpr int EPR = OUT == OUT_BF16 ? 2 : 1;  // elements per lane and row
+#pragma unroll 1
+                        for (int r0 = 0; r0 < 32; r0 += 8) {
+                            uint32_t x[8 * EPR];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int rr = row0 + r0 + i;
+                                const bool rv = rr < p.M && bb < p.batch_real;
+                                const long long rb = (long long)bb * p.stride_c + (long long)rr * p.ldc + colc;
+#pragma unroll
+                                for (int h = 0; h < EPR; ++h) {
+                                    const int e = (int)lane + 32 * h;
+                                    x[i * EPR + h] = 0u;
+                                    if (rv && colc + e < p.N) {
+                                        if constexpr (OUT == OUT_BF16)
+                                            x[i * EPR + h] = static_cast<const uint16_t*>(p.C)[rb + e];
+                                        else
+                                            x[i * EPR + h] = __float_as_uint(static_cast<const float*>(p.C)[rb + e]);
+                                    }
+                                }
+                            }
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int r = r0 + i;
+                                const uint32_t srow = sbuf + (uint32_t)r * 128u;
+#pragma unroll
+                                for (int h = 0; h < EPR; ++h) {
+                                    const int e = (int)lane + 32 * h;
+                                    if constexpr (OUT == OUT_BF16)
+                                        st_shared_u16(srow + ((uint32_t)((e >> 3) ^ (r & 7)) << 4) + (uint32_t)(e & 7) * 2u,
+                                                      (uint16_t)x[i * EPR + h]);
+                                    else
+                                        st_shared_u32(srow + ((uint32_t)((e >> 2) ^ (r & 7)) << 4) + (uint32_t)(e & 3) * 4u,
+                                                      x[i * EPR + h]);
+                                }
+                            }
+                        }
+                        __syncwarp();
+                        if (row_in) {
+                            const uint32_t srow = sbuf + lane * 128u;
+#pragma unroll
+                            for (int cc = 0; cc < 8; ++cc) {
+                                uint32_t x0, x1, x2, x3;
+                                ld_shared_v4(srow + ((uint32_t)(cc ^ (int)(lane & 7u)) << 4), x0, x1, x2, x3);
+                                const uint32_t xs[4] = {x0, x1, x2, x3};
+#pragma unroll
+                                for (int h = 0; h < 4; ++h) {
+                                    if constexpr (OUT == OUT_BF16) {
+                                        const int e = 8 * cc + 2 * h;
+                                        if (colc + e < p.N) v[e] = fmaf(p.beta, __uint_as_float(xs[h] << 16), v[e]);
+                                        if (colc + e + 1 < p.N)
+                                            v[e + 1] = fmaf(p.beta, __uint_as_float(xs[h] & 0xFFFF0000u), v[e + 1]);
+                                    } else {
+                                        const int e = 4 * cc + h;
+                                        if (colc + e < p.N) v[e] = fmaf(p.beta, __uint_as_float(xs[h]), v[e]);
+                                    }
+                                }
+                            }
+                        }
+                        __syncwarp();  // every lane has its C_in before the buffer is overwritten
+                    } else if (p.c_read && row_in) {
                         if (full_cols && p.c_tma) {
                             if constexpr (OUT == OUT_BF16) {
                                 const uint4* src = reinterpret_cast<const uint4*>(
@@ -509,20 +585,44 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
                             dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                    } else if (ARES == 0 && p.c_tma && colc + T::STG_COLS <= p.n_store_tma && bb < p.batch_real) {
-                        const uint32_t sbuf = stg + buf * T::STG_BYTES;
-                        if (lane == 0) bulk_wait_group_read<T::STG_BUFS - 1>();
-                        __syncwarp();
+                    } else if (ARES == 0) {
                         const uint32_t row_addr = sbuf + lane * 128u;
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
                             st_shared_v4(row_addr + ((uint32_t)(j ^ (int)(lane & 7u)) << 4), w[4 * j],
                                          w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_3d(&tmC, sbuf, colc, row0, bb);
-                            bulk_commit_group();
+                        if (tma_chunk) {
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_3d(&tmC, sbuf, colc, row0, bb);
+                                bulk_commit_group();
+                            }
+                        } else {
+                            // row by row: lane j writes element j (and j+32) of each row, coalesced
+                            __syncwarp();
+#pragma unroll 8
+                            for (int r = 0; r < 32; ++r) {
+                                const int rr = row0 + r;
+                                if (rr >= p.M || bb >= p.batch_real) continue;
+                                const long long rb = (long long)bb * p.stride_c + (long long)rr * p.ldc + colc;
+                                const uint32_t srow = sbuf + (uint32_t)r * 128u;
+                                if constexpr (OUT == OUT_BF16) {
+#pragma unroll
+                                    for (int h = 0; h < 2; ++h) {
+                                        const int e = (int)lane + 32 * h;
+                                        if (colc + e < p.N)
+                                            static_cast<uint16_t*>(p.C)[rb + e] = ld_shared_u16(
+                                                srow + ((uint32_t)((e >> 3) ^ (r & 7)) << 4) + (uint32_t)(e & 7) * 2u);
+                                    }
+                                } else {
+                                    const int e = (int)lane;
+                                    if (colc + e < p.N)
+                                        static_cast<float*>(p.C)[rb + e] = __uint_as_float(ld_shared_u32(
+                                            srow + ((uint32_t)((e >> 2) ^ (r & 7)) << 4) + (uint32_t)(e & 3) * 4u));
+                                }
+                            }
+                            __syncwarp();
                         }
                         if (T::STG_BUFS == 2) buf ^= 1;
                     } else if (row_in) {
@@ -585,10 +685,14 @@ __global__ void scale_c_kernel(TC* C, long long ldc, long long stride_c, int bat
 }
 
 // Copy a batch x rows x cols bf16 array into a buffer whose leading dimension is a multiple
-// of 8 elements and whose base is 16-byte aligned, so that TMA can read it.
+// of 8 elements and whose base is 16-byte aligned, so that TMA can read it.  Each thread writes
+// 8 elements with one 16-byte store.  Interior threads read the two aligned 16-byte words that
+// cover their (2-byte aligned) source window and realign them with byte permutes; threads whose
+// aligned window would reach outside [src_lo, src_hi) -- the source allocation's extent -- and
+// row tails use 2-byte loads.
 __global__ void pad_copy_kernel(const uint16_t* __restrict__ src, long long ld_src, long long bs_src,
                                 uint16_t* __restrict__ dst, long long ld_dst, long long bs_dst,
-                                int batch, int rows, int cols) {
+                                int batch, int rows, int cols, uintptr_t src_lo, uintptr_t src_hi) {
     const int vec_per_row = (cols + 7) >> 3;
     for (int b = blockIdx.z; b < batch; b += gridDim.z) {
         for (int r = blockIdx.y; r < rows; r += gridDim.y) {
@@ -598,10 +702,30 @@ __global__ void pad_copy_kernel(const uint16_t* __restrict__ src, long long ld_s
                  v += gridDim.x * blockDim.x) {
                 const int c = v << 3;
                 if (c + 8 <= cols) {
+                    const uintptr_t a = reinterpret_cast<uintptr_t>(s + c);
+                    const uintptr_t a0 = a & ~(uintptr_t)15;
+                    const uint32_t sh = (uint32_t)(a - a0);  // 0, 2, ..., 14
                     uint32_t e[4];
+                    if (a0 >= src_lo && a0 + 32 <= src_hi) {
+                        const uint4 lo = *reinterpret_cast<const uint4*>(a0);
+                        const uint4 hi = sh ? *reinterpret_cast<const uint4*>(a0 + 16) : lo;
+                        // y[j] = word (sh/4 + j) of the 32-byte window, selected without indexing
+                        const uint32_t wo = sh >> 2;
+                        const uint32_t y0 = wo == 0 ? lo.x : wo == 1 ? lo.y : wo == 2 ? lo.z : lo.w;
+                        const uint32_t y1 = wo == 0 ? lo.y : wo == 1 ? lo.z : wo == 2 ? lo.w : hi.x;
+                        const uint32_t y2 = wo == 0 ? lo.z : wo == 1 ? lo.w : wo == 2 ? hi.x : hi.y;
+                        const uint32_t y3 = wo == 0 ? lo.w : wo == 1 ? hi.x : wo == 2 ? hi.y : hi.z;
+                        const uint32_t y4 = wo == 0 ? hi.x : wo == 1 ? hi.y : wo == 2 ? hi.z : hi.w;
+                        const uint32_t sel = (sh & 2) ? 0x5432u : 0x3210u;  // half-word shift or none
+                        e[0] = __byte_perm(y0, y1, sel);
+                        e[1] = __byte_perm(y1, y2, sel);
+                        e[2] = __byte_perm(y2, y3, sel);
+                        e[3] = __byte_perm(y3, y4, sel);
+                    } else {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        e[j] = (uint32_t)s[c + 2 * j] | ((uint32_t)s[c + 2 * j + 1] << 16);
+                        for (int j = 0; j < 4; ++j)
+                            e[j] = (uint32_t)s[c + 2 * j] | ((uint32_t)s[c + 2 * j + 1] << 16);
+                    }
                     *reinterpret_cast<uint4*>(d + c) = make_uint4(e[0], e[1], e[2], e[3]);
                 } else {
                     for (int j = c; j < cols; ++j) d[j] = s[j];
