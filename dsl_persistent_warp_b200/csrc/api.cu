@@ -112,6 +112,14 @@ int pack_factor(const PlanDesc& pd, bool b_mn, int N) {
 
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
+// Failure-detection test hook: with GEMM_BF16_TEST_STALL_LOADS=1 the kernel's producer issues
+// no loads, so the MMA thread's first bounded wait expires and the kernel reports a timeout
+// through gemm_bf16_device_status.  Nothing faults; the context stays usable.
+bool test_stall_requested() {
+    const char* e = std::getenv("GEMM_BF16_TEST_STALL_LOADS");
+    return e && e[0] == '1';
+}
+
 // m-blocks per raster group; GEMM_BF16_GROUP_M (1..64) overrides the default for tuning sweeps.
 int group_m() {
     const char* e = std::getenv("GEMM_BF16_GROUP_M");
@@ -410,6 +418,7 @@ gemm_status_t run(Req r) {
         p.n_store_tma = ((long long)r.N * es) % 16 == 0 ? (int)round_up(r.N, stg_cols) : r.N;
         p.c_read = r.beta != 0.0f ? 1 : 0;
         p.timeout_ns = g_timeout_ns.load();
+        p.test_stall = test_stall_requested() ? 1 : 0;
         st = launch_by_plan(plan, r.b_mn, r.out, ma, mb, mc, p, dev, di.sms, r.stream);
     }
     if (ws) cudaFreeAsync(ws, r.stream);

@@ -65,6 +65,8 @@ struct KParams {
     int pack;                // batch entries side by side in one tile (MN-major B; 1 = none):
                              // tile column c belongs to entry nb*pack + c/N, column c%N
     int batch_real;          // number of batch entries (p.batch counts tile batches)
+    int test_stall;          // test hook: the producer issues nothing, so the first bounded
+                             // wait of the MMA thread expires (failure-detection tests)
     unsigned long long timeout_ns;
 };
 
@@ -240,8 +242,8 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             const uint64_t pol = l2_policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
-            bool ok = true;
-            if constexpr (ARES != 0) {
+            bool ok = p.test_stall == 0;
+            if (ARES != 0 && ok) {
                 // This CTA's 128 rows of the single M tile, every k-block, once.
                 if (rank == 0) mbar_arrive_expect_tx(bar_ares, (uint32_t)(T::A_BYTES * CG * p.k_blocks));
                 const uint32_t ares_bar = CG == 2 ? map_to_rank(bar_ares, 0) : bar_ares;
