@@ -70,6 +70,36 @@ bool device_info(int dev, DevInfo& out) {
     return true;
 }
 
+// Stream-ordered pool of the library's per-call workspace (alignment pre-pass copies, split-K
+// partial sums and counters), one per device.  Its release threshold is unlimited: memory freed
+// at the end of a call stays in the pool for the next call on any stream instead of going back
+// to the driver at the next synchronisation, so steady-state calls map no new pages.  The pool
+// holds the largest workspace seen so far until the process exits.
+std::mutex g_pool_mu;
+std::array<cudaMemPool_t, kMaxDevices> g_pool{};
+
+gemm_status_t workspace_pool(int dev, cudaMemPool_t* out) {
+    if (dev < 0 || dev >= kMaxDevices) return GEMM_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_pool_mu);
+    if (g_pool[dev] == nullptr) {
+        cudaMemPoolProps props;
+        std::memset(&props, 0, sizeof props);
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return GEMM_ERR_CUDA;
+        uint64_t keep = UINT64_MAX;
+        if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+            cudaMemPoolDestroy(pool);
+            return GEMM_ERR_CUDA;
+        }
+        g_pool[dev] = pool;
+    }
+    *out = g_pool[dev];
+    return GEMM_OK;
+}
+
 // One request, in the batched form (batch == 1 for the plain GEMM).
 struct Req {
     int batch, M, N, K;
@@ -168,9 +198,24 @@ gemm_status_t encode_3d(CUtensorMap* m, const void* base, bool f32, uint64_t d0,
 }
 
 // Sustained rate of each plan with every SM busy (TFLOP/s measured on B200, 8192^3 bf16); only
-// the ratios matter.  The automatic choice minimises  waves * tile_flops / per-cluster rate:
+// the ratios matter.  The automatic choice minimises the modelled time of plan_time() below:
 // large tiles move fewer operand bytes per FLOP, small tiles quantise better on small grids.
 constexpr double kPlanRate[kNumStreamPlans] = {880.0, 1190.0, 1250.0, 790.0, 1400.0};
+
+// Split-K limits: at most kMaxSplits slices of K, each at least kMinSplitKBlocks k-blocks long
+// (the smem ring needs a few blocks to fill), and a split must beat the unsplit choice by 10%.
+constexpr int kMaxSplits = 8;
+constexpr int kMinSplitKBlocks = 8;
+// Operand bytes one CTA pulls through TMA per second when its tiles are not compute-bound
+// (measured on B200 with few, deep tiles: 8192x256x4096, 1024x1024x8192).
+constexpr double kCtaOperandBytesPerSec = 140e9;
+// Split-K cost per unit, measured on B200: a fixed part (counter, fences, the longer fixup
+// epilogue), the write of the unit's fp32 partial sums and the last unit's read of the others.
+constexpr double kSplitFixedSec = 4e-6;
+constexpr double kSplitWriteBytesPerSec = 45e9;
+constexpr double kSplitReadBytesPerSec = 90e9;
+// Split-K arrival counters per CTA and tile: one per epilogue warp.
+constexpr int kSplitCountersPerCta = 4;
 
 // Can plan `i` serve this request?
 bool plan_serves(int i, const Req& r) {
@@ -179,27 +224,92 @@ bool plan_serves(int i, const Req& r) {
     return true;
 }
 
-// Plan for a request on a device with `sms` SMs (auto unless overridden).
-int choose_plan(const Req& r, int sms) {
+// Output tiles of plan `pd` for the request.
+long long plan_tiles(const PlanDesc& pd, const Req& r) {
+    const long long tm = 128LL * pd.cg, tn = (long long)pd.bn * pd.nsub;
+    const int pk = pack_factor(pd, r.b_mn, r.N);
+    return pk > 1 ? cdiv(r.M, tm) * cdiv(r.batch, pk) : cdiv(r.M, tm) * cdiv(r.N, tn) * r.batch;
+}
+
+// Modelled time (s) of streaming plan `i` with K cut into `splits` slices: waves of work units,
+// each bound by the plan's per-cluster tensor rate or by its CTAs' operand streaming, plus,
+// when split, each unit's partial-sum write and the last unit's read of the other slices.
+double plan_time(int i, const Req& r, int sms, int splits) {
+    const PlanDesc& pd = kPlans[i];
+    const long long tm = 128LL * pd.cg, tn = (long long)pd.bn * pd.nsub;
+    const long long slots = sms / pd.cg;
+    const long long kb = cdiv(cdiv(r.K, pd.bk), splits);  // k-blocks per unit
+    const double unit_k = (double)(kb * pd.bk);
+    const double compute = 2.0 * (double)(tm * tn) * unit_k / (kPlanRate[i] * 1e12 / (double)slots);
+    const double stream = (double)(tm + tn) * unit_k * 2.0 / (pd.cg * kCtaOperandBytesPerSec);
+    double t = (double)cdiv(plan_tiles(pd, r) * splits, slots) * (compute > stream ? compute : stream);
+    if (splits > 1) {
+        const double partial = 128.0 * (double)tn * 4.0;  // bytes per CTA and unit
+        t += kSplitFixedSec + partial / kSplitWriteBytesPerSec + (splits - 1) * partial / kSplitReadBytesPerSec;
+    }
+    return t;
+}
+
+// Split counts the kernel takes for plan `pd`: every slice non-empty and the same length
+// except the last.
+bool split_valid(const PlanDesc& pd, const Req& r, int splits) {
+    if (splits == 1) return true;
+    if (pd.ares || splits < 1 || splits > kMaxSplits) return false;
+    const long long kb = cdiv(r.K, pd.bk);
+    return cdiv(kb, cdiv(kb, splits)) == splits;
+}
+
+// GEMM_BF16_SPLIT_K=s (1..8) forces s slices of K wherever the plan takes it (tests, tuning);
+// unset or 0 leaves the choice to the model.
+int forced_splits() {
+    const char* e = std::getenv("GEMM_BF16_SPLIT_K");
+    if (e) {
+        const int v = std::atoi(e);
+        if (v >= 1 && v <= kMaxSplits) return v;
+    }
+    return 0;
+}
+
+struct Choice {
+    int plan;
+    int splits;
+};
+
+// Plan and K split for a request on a device with `sms` SMs (auto unless overridden); without
+// `allow_split` the best unsplit plan.
+Choice choose(const Req& r, int sms, bool allow_split) {
+    const int fs = allow_split ? forced_splits() : 1;
     const int forced = g_plan_override.load();
-    if (forced >= 0 && plan_serves(forced, r)) return forced;
-    // Shared-W batched shapes with short K are bound by streaming X and Y through HBM: the
-    // 256x256 tile holding several batch entries side by side measured fastest (W re-reads hit
-    // L2); the resident-W plans (5-7) stay available through gemm_bf16_set_plan.
-    if (r.b_mn && r.K <= 1024 && pack_factor(kPlans[2], r.b_mn, r.N) > 1) return 2;
-    int best = 0;
+    int lo = 0, hi = kNumStreamPlans - 1;
+    if (forced >= 0 && plan_serves(forced, r)) {
+        if (kPlans[forced].ares) return {forced, 1};
+        lo = hi = forced;
+    } else if (r.b_mn && r.K <= 1024 && pack_factor(kPlans[2], r.b_mn, r.N) > 1) {
+        // Shared-W batched shapes with short K are bound by streaming X and Y through HBM: the
+        // 256x256 tile holding several batch entries side by side measured fastest (W re-reads
+        // hit L2); the resident-W plans (5-7) stay available through gemm_bf16_set_plan.
+        lo = hi = 2;
+    }
+    Choice best{lo, 1};
     double best_t = 0.0;
-    for (int i = 0; i < kNumStreamPlans; ++i) {
+    bool have = false;
+    for (int i = lo; i <= hi; ++i) {
         const PlanDesc& pd = kPlans[i];
-        const long long tm = 128LL * pd.cg, tn = (long long)pd.bn * pd.nsub;
-        const int pk = pack_factor(pd, r.b_mn, r.N);
-        const long long tiles = pk > 1 ? cdiv(r.M, tm) * cdiv(r.batch, pk) : cdiv(r.M, tm) * cdiv(r.N, tn) * r.batch;
-        const long long slots = sms / pd.cg;
-        const long long waves = cdiv(tiles, slots);
-        const double t = (double)waves * (double)(tm * tn) * (double)slots / kPlanRate[i];
-        if (i == 0 || t < best_t * 0.999) {
-            best = i;
-            best_t = t;
+        const long long kb = cdiv(r.K, pd.bk);
+        if (fs > 0) {
+            const int s = split_valid(pd, r, fs) ? fs : 1;
+            const double t = plan_time(i, r, sms, s);
+            if (!have || t < best_t * 0.999) best = {i, s}, best_t = t, have = true;
+            continue;
+        }
+        long long smax = kb / kMinSplitKBlocks;
+        if (pd.ares || smax < 1 || !allow_split) smax = 1;
+        if (smax > kMaxSplits) smax = kMaxSplits;
+        for (int s = 1; s <= (int)smax; ++s) {
+            if (!split_valid(pd, r, s)) continue;
+            const double t = plan_time(i, r, sms, s);
+            const double margin = s == 1 ? 0.999 : 0.90;
+            if (!have || t < best_t * margin) best = {i, s}, best_t = t, have = true;
         }
     }
     return best;
@@ -210,6 +320,7 @@ gemm_status_t launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, co
                                 const KParams& p, int dev, int sms, cudaStream_t stream) {
     using T = Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES>;
     auto kern = gemm_persistent<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES>;
+    static_assert(T::EPI_WARPS == kSplitCountersPerCta, "split-K counters sized per epilogue warp");
     static std::array<std::atomic<int>, kMaxDevices> attr_done{};
     static std::array<std::atomic<int>, kMaxDevices> max_clusters{};
     if (!attr_done[dev].load()) {
@@ -236,7 +347,8 @@ gemm_status_t launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, co
         max_clusters[dev].store(clusters);
         attr_done[dev].store(1);
     }
-    const int clusters = (int)(p.tiles < max_clusters[dev].load() ? p.tiles : max_clusters[dev].load());
+    const long long units = (long long)p.tiles * (p.splits > 1 ? p.splits : 1);  // work units
+    const int clusters = (int)(units < max_clusters[dev].load() ? units : max_clusters[dev].load());
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(clusters * CG, 1, 1);
     cfg.blockDim = dim3(T::THREADS, 1, 1);
@@ -348,9 +460,31 @@ gemm_status_t run(Req r) {
         sb_p = b_rows * ldb_p;
         ws_b = (size_t)round_up(sb_p * 2 * r.batch, 256);
     }
+    // Split-K partial sums (fp32, one 128 x tile_n slab per CTA, tile and slice) and the
+    // per-(tile, CTA, epilogue warp) arrival counters, which must start at zero.
+    const Choice ch = choose(r, di.sms, true);
+    const int plan = ch.plan;
+    const PlanDesc pd = kPlans[plan];
+    const long long tiles_est = plan_tiles(pd, r);
+    size_t ws_p = 0, ws_n = 0;
+    if (ch.splits > 1) {
+        ws_p = (size_t)tiles_est * pd.cg * ch.splits * 128 * pd.bn * pd.nsub * sizeof(float);
+        ws_n = (size_t)round_up(tiles_est * pd.cg * kSplitCountersPerCta * (long long)sizeof(unsigned int), 256);
+    }
     void* ws = nullptr;
-    if (ws_a + ws_b) {
-        if (cudaMallocAsync(&ws, ws_a + ws_b, r.stream) != cudaSuccess) return GEMM_ERR_NO_MEMORY;
+    if (ws_a + ws_b + ws_p + ws_n) {
+        cudaMemPool_t pool = nullptr;
+        const gemm_status_t ps = workspace_pool(dev, &pool);
+        if (ps != GEMM_OK) return ps;
+        if (cudaMallocFromPoolAsync(&ws, ws_a + ws_b + ws_p + ws_n, pool, r.stream) != cudaSuccess)
+            return GEMM_ERR_NO_MEMORY;
+    }
+    float* ws_partials = ch.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + ws_a + ws_b) : nullptr;
+    unsigned int* ws_counters =
+        ch.splits > 1 ? reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + ws_a + ws_b + ws_p) : nullptr;
+    if (ws_n && cudaMemsetAsync(ws_counters, 0, ws_n, r.stream) != cudaSuccess) {
+        cudaFreeAsync(ws, r.stream);
+        return GEMM_ERR_CUDA;
     }
     const void* A = r.A;
     const void* B = r.B;
@@ -364,8 +498,6 @@ gemm_status_t run(Req r) {
         B = dst;
     }
 
-    const int plan = choose_plan(r, di.sms);
-    const PlanDesc pd = kPlans[plan];
     const int b_chunk = pd.bn * pd.nsub / pd.cg;  // B rows per CTA and stage
     const int es = r.out == OUT_F32 ? 4 : 2;
     const int stg_cols = r.out == OUT_F32 ? 32 : 64;
@@ -406,6 +538,12 @@ gemm_status_t run(Req r) {
         }
         p.tiles = p.m_blocks * p.n_blocks * p.batch;
         p.k_blocks = (int)cdiv(r.K, pd.bk);
+        if (ch.splits > 1) {
+            p.splits = ch.splits;
+            p.kb_per_split = (int)cdiv(p.k_blocks, ch.splits);
+            p.ws = ws_partials;
+            p.counters = ws_counters;
+        }
         p.group_m = group_m();
         p.alpha = r.alpha;
         p.beta = r.beta;
@@ -507,7 +645,7 @@ gemm_status_t run_noalloc(Req r) {
         }
     }
 
-    const int plan = choose_plan(r, di.sms);
+    const int plan = choose(r, di.sms, false).plan;
     const PlanDesc pd = kPlans[plan];
     const int b_chunk = pd.bn * pd.nsub / pd.cg;  // B rows per CTA and stage
     const int es = r.out == OUT_F32 ? 4 : 2;

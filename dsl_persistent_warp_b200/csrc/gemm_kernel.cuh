@@ -65,6 +65,13 @@ struct KParams {
     int pack;                // batch entries side by side in one tile (MN-major B; 1 = none):
                              // tile column c belongs to entry nb*pack + c/N, column c%N
     int batch_real;          // number of batch entries (p.batch counts tile batches)
+    int splits;              // K slices per tile (split-K; <= 1: none).  Work unit u covers tile
+                             // u / splits and k-blocks [s*kb_per_split, (s+1)*kb_per_split), s = u % splits
+    int kb_per_split;
+    float* ws;               // split-K partials: per (tile, CTA rank, slice) the CTA's 128 rows x
+                             // TILE_N columns in fp32, column-major (element (r, c) at c*128 + r)
+    unsigned int* counters;  // split-K arrivals per (tile, CTA rank, epilogue warp); zero on entry,
+                             // and the last arrival puts it back to zero
     int test_stall;          // test hook: the producer issues nothing, so the first bounded
                              // wait of the MMA thread expires (failure-detection tests)
     unsigned long long timeout_ns;
@@ -253,11 +260,15 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     else tma_load_3d_pair(sa, &tmA, ares_bar, kb * T::BK, (int)rank * 128, 0, pol);
                 }
             }
-            for (int t = cluster_id; ok && t < p.tiles; t += num_clusters) {
+            const int S = (ARES == 0 && p.splits > 1) ? p.splits : 1;  // split-K: streaming plans only
+            for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters) {
+                const int t = u / S;
+                const int kb_lo = S > 1 ? (u % S) * p.kb_per_split : 0;
+                const int kb_hi = S > 1 ? min(p.k_blocks, kb_lo + p.kb_per_split) : p.k_blocks;
                 int b, mb, nb;
                 decode_tile(p, t, b, mb, nb);
                 const int a_row = mb * T::BM + (int)rank * 128;
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!wait_phase<CG, false>(bar_empty(stage), phase ^ 1u, slot_abort, rank,
                                                p.timeout_ns, kStatusProducer)) {
                         ok = false;
@@ -320,8 +331,11 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 ok = wait_phase<CG, false>(bar_ares, 0u, slot_abort, rank, p.timeout_ns, kStatusMma);
                 tc_fence_after();
             }
-            for (int t = cluster_id; ok && t < p.tiles; t += num_clusters) {
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
+            const int S = (ARES == 0 && p.splits > 1) ? p.splits : 1;  // split-K: streaming plans only
+            for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters) {
+                const int kb_lo = S > 1 ? (u % S) * p.kb_per_split : 0;
+                const int kb_hi = S > 1 ? min(p.k_blocks, kb_lo + p.kb_per_split) : p.k_blocks;
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, rank, p.timeout_ns,
                                                kStatusMma)) {
                         ok = false;
@@ -334,7 +348,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
 #pragma unroll
                     for (int sub = 0; sub < NSUB; ++sub) {
                         const int slot = NSUB == 1 ? acc : sub;
-                        if (kb == 0) {
+                        if (kb == kb_lo) {
                             // the slot must have been drained by the epilogue of its last use
                             if (!wait_phase<CG, CG == 2>(bar_tempty(slot), ((tph >> slot) & 1u) ^ 1u, slot_abort, rank,
                                                          p.timeout_ns, kStatusMma)) {
@@ -350,9 +364,9 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                             // K=16 step: 32 bytes along a K-major row; 16 rows (2 KiB) of an MN-major box
                             const uint64_t adesc = a_st + (uint64_t)((kk * 32) >> 4);
                             const uint64_t bdesc = b_sub + (uint64_t)((B_MN ? kk * 2048 : kk * 32) >> 4);
-                            umma_f16<CG>(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                            umma_f16<CG>(d_tmem, adesc, bdesc, IDESC, (kb != kb_lo || kk != 0) ? 1u : 0u);
                         }
-                        if (kb == p.k_blocks - 1) {
+                        if (kb == kb_hi - 1) {
                             // accumulator of this slot complete: hand it to the epilogue
                             if constexpr (CG == 1) {
                                 umma_commit<1>(bar_tfull(slot));
@@ -394,11 +408,264 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         int acc = 0;
         int buf = 0;
         bool ok = true;
-        for (int t = cluster_id; ok && t < p.tiles; t += num_clusters) {
+        // alpha/beta, conversion and store of chunk c (STG_COLS columns) of sub-tile `sub` of the
+        // tile (b, nb) for the 32-row slab starting at row0; v holds this lane's row.
+        auto finish_chunk = [&](int b, int nb, int row0, int row, int sub, int c, float (&v)[T::STG_COLS]) {
+            const int col_tile = sub * T::BN_CTA;  // column within the tile
+            const int jc = c * T::STG_COLS;
+            const int tcol = col_tile + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
+            const int bb = p.pack > 1 ? nb * p.pack + tcol / p.N : b;
+            const int colc = p.pack > 1 ? tcol % p.N : nb * T::TILE_N + tcol;
+            const long long cbase = (long long)bb * p.stride_c + (long long)row * p.ldc;
+            const bool row_in = row < p.M && bb < p.batch_real;
+            const bool full_cols = colc + T::STG_COLS <= p.N;
+            // A chunk goes out as one tensor store when C is TMA-addressable up to the
+            // chunk's end; otherwise (unaligned ldc, a ragged right edge) the warp moves it
+            // row by row through the staging buffer so that every access is coalesced.
+            const bool tma_chunk =
+                ARES == 0 && p.c_tma && colc + T::STG_COLS <= p.n_store_tma && bb < p.batch_real;
+            const bool coop_chunk = ARES == 0 && !tma_chunk;
+            const uint32_t sbuf = stg + buf * T::STG_BYTES;
+            if (ARES == 0) {
+                // the buffer may still be read by an earlier tensor store
+                if (lane == 0) bulk_wait_group_read<T::STG_BUFS - 1>();
+                __syncwarp();
+            }
+#pragma unroll
+            for (int j = 0; j < T::STG_COLS; ++j) v[j] *= p.alpha;
+            if (p.c_read && coop_chunk) {
+                // C_in: lane j reads elements j (and j+32 for bf16) of each of the warp's 32
+                // rows; element e of row r sits in 16-byte chunk (e*ES/16) ^ (r & 7).  Rows
+                // go 8 at a time so that 8 (16 for bf16) loads per lane are in flight.
+                constexpr int EPR = OUT == OUT_BF16 ? 2 : 1;  // elements per lane and row
+#pragma unroll 1
+                for (int r0 = 0; r0 < 32; r0 += 8) {
+                    uint32_t x[8 * EPR];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int rr = row0 + r0 + i;
+                        const bool rv = rr < p.M && bb < p.batch_real;
+                        const long long rb = (long long)bb * p.stride_c + (long long)rr * p.ldc + colc;
+#pragma unroll
+                        for (int h = 0; h < EPR; ++h) {
+                            const int e = (int)lane + 32 * h;
+                            x[i * EPR + h] = 0u;
+                            if (rv && colc + e < p.N) {
+                                if constexpr (OUT == OUT_BF16)
+                                    x[i * EPR + h] = static_cast<const uint16_t*>(p.C)[rb + e];
+                                else
+                                    x[i * EPR + h] = __float_as_uint(static_cast<const float*>(p.C)[rb + e]);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = r0 + i;
+                        const uint32_t srow = sbuf + (uint32_t)r * 128u;
+#pragma unroll
+                        for (int h = 0; h < EPR; ++h) {
+                            const int e = (int)lane + 32 * h;
+                            if constexpr (OUT == OUT_BF16)
+                                st_shared_u16(srow + ((uint32_t)((e >> 3) ^ (r & 7)) << 4) + (uint32_t)(e & 7) * 2u,
+                                              (uint16_t)x[i * EPR + h]);
+                            else
+                                st_shared_u32(srow + ((uint32_t)((e >> 2) ^ (r & 7)) << 4) + (uint32_t)(e & 3) * 4u,
+                                              x[i * EPR + h]);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (row_in) {
+                    const uint32_t srow = sbuf + lane * 128u;
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        uint32_t x0, x1, x2, x3;
+                        ld_shared_v4(srow + ((uint32_t)(cc ^ (int)(lane & 7u)) << 4), x0, x1, x2, x3);
+                        const uint32_t xs[4] = {x0, x1, x2, x3};
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            if constexpr (OUT == OUT_BF16) {
+                                const int e = 8 * cc + 2 * h;
+                                if (colc + e < p.N) v[e] = fmaf(p.beta, __uint_as_float(xs[h] << 16), v[e]);
+                                if (colc + e + 1 < p.N)
+                                    v[e + 1] = fmaf(p.beta, __uint_as_float(xs[h] & 0xFFFF0000u), v[e + 1]);
+                            } else {
+                                const int e = 4 * cc + h;
+                                if (colc + e < p.N) v[e] = fmaf(p.beta, __uint_as_float(xs[h]), v[e]);
+                            }
+                        }
+                    }
+                }
+                __syncwarp();  // every lane has its C_in before the buffer is overwritten
+            } else if (p.c_read && row_in) {
+                if (full_cols && p.c_tma) {
+                    if constexpr (OUT == OUT_BF16) {
+                        const uint4* src = reinterpret_cast<const uint4*>(
+                            static_cast<const uint16_t*>(p.C) + cbase + colc);
+#pragma unroll
+                        for (int j = 0; j < T::STG_COLS / 8; ++j) {
+                            const uint4 w = src[j];
+                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                v[8 * j + 2 * h] =
+                                    fmaf(p.beta, __uint_as_float(ww[h] << 16), v[8 * j + 2 * h]);
+                                v[8 * j + 2 * h + 1] = fmaf(
+                                    p.beta, __uint_as_float(ww[h] & 0xFFFF0000u), v[8 * j + 2 * h + 1]);
+                            }
+                        }
+                    } else {
+                        const float4* src = reinterpret_cast<const float4*>(
+                            static_cast<const float*>(p.C) + cbase + colc);
+#pragma unroll
+                        for (int j = 0; j < T::STG_COLS / 4; ++j) {
+                            const float4 w = src[j];
+                            v[4 * j + 0] = fmaf(p.beta, w.x, v[4 * j + 0]);
+                            v[4 * j + 1] = fmaf(p.beta, w.y, v[4 * j + 1]);
+                            v[4 * j + 2] = fmaf(p.beta, w.z, v[4 * j + 2]);
+                            v[4 * j + 3] = fmaf(p.beta, w.w, v[4 * j + 3]);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < T::STG_COLS; ++j) {
+                        if (colc + j < p.N) {
+                            float cin;
+                            if constexpr (OUT == OUT_BF16)
+                                cin = __uint_as_float(
+                                    (uint32_t)(static_cast<const uint16_t*>(p.C)[cbase + colc + j]) << 16);
+                            else
+                                cin = static_cast<const float*>(p.C)[cbase + colc + j];
+                            v[j] = fmaf(p.beta, cin, v[j]);
+                        }
+                    }
+                }
+            }
+            // pack the 128-byte row segment into 8 x 16-byte words
+            uint32_t w[32];
+            if constexpr (OUT == OUT_BF16) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
+            }
+            if (ARES != 0 && p.c_tma && full_cols && row_in) {
+                // whole 128-byte row segment of this thread, inside N: eight 16-byte stores
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<char*>(p.C) +
+                                                      (cbase + colc) * (OUT == OUT_BF16 ? 2 : 4));
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+            } else if (ARES == 0) {
+                const uint32_t row_addr = sbuf + lane * 128u;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    st_shared_v4(row_addr + ((uint32_t)(j ^ (int)(lane & 7u)) << 4), w[4 * j],
+                                 w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                if (tma_chunk) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tmC, sbuf, colc, row0, bb);
+                        bulk_commit_group();
+                    }
+                } else {
+                    // row by row: lane j writes element j (and j+32) of each row, coalesced
+                    __syncwarp();
+#pragma unroll 8
+                    for (int r = 0; r < 32; ++r) {
+                        const int rr = row0 + r;
+                        if (rr >= p.M || bb >= p.batch_real) continue;
+                        const long long rb = (long long)bb * p.stride_c + (long long)rr * p.ldc + colc;
+                        const uint32_t srow = sbuf + (uint32_t)r * 128u;
+                        if constexpr (OUT == OUT_BF16) {
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const int e = (int)lane + 32 * h;
+                                if (colc + e < p.N)
+                                    static_cast<uint16_t*>(p.C)[rb + e] = ld_shared_u16(
+                                        srow + ((uint32_t)((e >> 3) ^ (r & 7)) << 4) + (uint32_t)(e & 7) * 2u);
+                            }
+                        } else {
+                            const int e = (int)lane;
+                            if (colc + e < p.N)
+                                static_cast<float*>(p.C)[rb + e] = __uint_as_float(ld_shared_u32(
+                                    srow + ((uint32_t)((e >> 2) ^ (r & 7)) << 4) + (uint32_t)(e & 3) * 4u));
+                        }
+                    }
+                    __syncwarp();
+                }
+                if (T::STG_BUFS == 2) buf ^= 1;
+            } else if (row_in) {
+                if constexpr (OUT == OUT_BF16) {
+                    uint16_t* dst = static_cast<uint16_t*>(p.C) + cbase + colc;
+#pragma unroll
+                    for (int j = 0; j < T::STG_COLS; ++j)
+                        if (colc + j < p.N)
+                            dst[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
+                } else {
+                    float* dst = static_cast<float*>(p.C) + cbase + colc;
+#pragma unroll
+                    for (int j = 0; j < T::STG_COLS; ++j)
+                        if (colc + j < p.N) dst[j] = __uint_as_float(w[j]);
+                }
+            }
+        };
+        // TMEM -> registers: chunk c (STG_COLS columns) of the slot whose lane-quarter row is trow.
+        auto load_chunk = [&](uint32_t trow, int c, float (&v)[T::STG_COLS]) {
+            uint32_t r0[32];
+            tmem_ld_32x32b_x32(trow + c * T::STG_COLS, r0);
+            if constexpr (OUT == OUT_BF16) {
+                uint32_t r1[32];
+                tmem_ld_32x32b_x32(trow + c * T::STG_COLS + 32, r1);
+                tmem_ld_wait(r0);
+                tmem_ld_wait(r1);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[32 + j] = __uint_as_float(r1[j]);
+            } else {
+                tmem_ld_wait(r0);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
+        };
+        // Split-K partial sums travel as 4 KiB pieces: 32 rows x 32 fp32 columns, held in global
+        // memory as the image of the staging buffer (row r at byte 128 r, 16-byte word w of the
+        // row at ((w ^ (r & 7)) << 4)).  Moving a piece through the buffer turns the
+        // lane-per-row layout of TMEM into 512-byte coalesced accesses.
+        constexpr int PIECES = T::STG_COLS / 32;               // pieces per chunk
+        constexpr int WS_TILE = 128 * NSUB * BN;               // floats per (tile, CTA rank, slice)
+        constexpr int WS_WARP = WS_TILE / T::EPI_WARPS;        // floats per epilogue warp
+        auto put_piece = [&](float* g, const float* x, uint32_t sb) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                st_shared_v4(sb + lane * 128u + ((uint32_t)(j ^ (int)(lane & 7u)) << 4), __float_as_uint(x[4 * j]),
+                             __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
+                             __float_as_uint(x[4 * j + 3]));
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                uint32_t x0, x1, x2, x3;
+                ld_shared_v4(sb + (uint32_t)i * 512u + lane * 16u, x0, x1, x2, x3);
+                reinterpret_cast<uint4*>(g)[i * 32 + (int)lane] = make_uint4(x0, x1, x2, x3);
+            }
+            __syncwarp();
+        };
+        const int S = (ARES == 0 && p.splits > 1) ? p.splits : 1;  // split-K: streaming plans only
+        for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters) {
+            const int t = u / S;
+            const int sl = u % S;
             int b, mb, nb;
             decode_tile(p, t, b, mb, nb);
             const int row0 = mb * T::BM + (int)rank * 128 + 32 * q;
             const int row = row0 + (int)lane;
+            // this warp's partials of slice s of the tile: pieces in (sub, ci, piece) order
+            auto slab = [&](int s) { return p.ws + ((size_t)(t * CG + (int)rank) * S + s) * WS_TILE + (size_t)ew * WS_WARP; };
+            if (S > 1) {
+                // the staging buffer must not be read by a tensor store still in flight
+                if (lane == 0) bulk_wait_group_read<0>();
+                __syncwarp();
+            }
             for (int sub = 0; sub < NSUB; ++sub) {
                 const int slot = NSUB == 1 ? acc : sub;
                 int w_ok = 1;
@@ -413,234 +680,106 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 tc_fence_after();
                 tph ^= 1u << slot;
                 const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(slot * BN);
-                // MMA column j of sub-tile `sub` comes from CTA q = j / BN_CTA's B chunk, row
-                // sub*BN_CTA + j % BN_CTA of it, i.e. tile column q*B_CHUNK + sub*BN_CTA + j % BN_CTA.
-                const int col_tile = sub * T::BN_CTA;  // column within the tile
 #pragma unroll 1
                 for (int ci = 0; ci < CPW; ++ci) {
                     const int c = half * CPW + ci;
                     float v[T::STG_COLS];
-                    {
-                        uint32_t r0[32];
-                        tmem_ld_32x32b_x32(trow + c * T::STG_COLS, r0);
-                        if constexpr (OUT == OUT_BF16) {
-                            uint32_t r1[32];
-                            tmem_ld_32x32b_x32(trow + c * T::STG_COLS + 32, r1);
-                            tmem_ld_wait(r0);
-                            tmem_ld_wait(r1);
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[32 + j] = __uint_as_float(r1[j]);
-                        } else {
-                            tmem_ld_wait(r0);
+                    load_chunk(trow, c, v);
+                    if (S == 1) {
+                        if (ci == CPW - 1) {
+                            // Slot drained: hand it back to the MMA warp (leader CTA).
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * slot);
                         }
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
-                    }
-                    if (ci == CPW - 1) {
-                        // Slot drained: hand it back to the MMA warp (leader CTA).
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * slot);
-                    }
-                    const int jc = c * T::STG_COLS;
-                    const int tcol = col_tile + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
-                    const int bb = p.pack > 1 ? nb * p.pack + tcol / p.N : b;
-                    const int colc = p.pack > 1 ? tcol % p.N : nb * T::TILE_N + tcol;
-                    const long long cbase = (long long)bb * p.stride_c + (long long)row * p.ldc;
-                    const bool row_in = row < p.M && bb < p.batch_real;
-                    const bool full_cols = colc + T::STG_COLS <= p.N;
-                    // A chunk goes out as one tensor store when C is TMA-addressable up to the
-                    // chunk's end; otherwise (unaligned ldc, a ragged right edge) the warp moves it
-                    // row by row through the staging buffer so that every access is coalesced.
-                    const bool tma_chunk =
-                        ARES == 0 && p.c_tma && colc + T::STG_COLS <= p.n_store_tma && bb < p.batch_real;
-                    const bool coop_chunk = ARES == 0 && !tma_chunk;
-                    const uint32_t sbuf = stg + buf * T::STG_BYTES;
-                    if (ARES == 0) {
-                        // the buffer may still be read by an earlier tensor store
-                        if (lane == 0) bulk_wait_group_read<T::STG_BUFS - 1>();
-                        __syncwarp();
-                    }
-#pragma unroll
-                    for (int j = 0; j < T::STG_COLS; ++j) v[j] *= p.alpha;
-                    if (p.c_read && coop_chunk) {
-                        // C_in: lane j reads elements j (and j+32 for bf16) of each of the warp's 32
-                        // rows; element e of row r sits in 16-byte chunk (e*ES/16) ^ (r & 7).  Rows
-                        // go 8 at a time so that 8 (16 for bf16) loads per lane are in flight.
-                        constexpr int EPR = OUT == OUT_BF16 ? 2 : 1;  // elements per lane and row
-#pragma unroll 1
-                        for (int r0 = 0; r0 < 32; r0 += 8) {
-                            uint32_t x[8 * EPR];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int rr = row0 + r0 + i;
-                                const bool rv = rr < p.M && bb < p.batch_real;
-                                const long long rb = (long long)bb * p.stride_c + (long long)rr * p.ldc + colc;
-#pragma unroll
-                                for (int h = 0; h < EPR; ++h) {
-                                    const int e = (int)lane + 32 * h;
-                                    x[i * EPR + h] = 0u;
-                                    if (rv && colc + e < p.N) {
-                                        if constexpr (OUT == OUT_BF16)
-                                            x[i * EPR + h] = static_cast<const uint16_t*>(p.C)[rb + e];
-                                        else
-                                            x[i * EPR + h] = __float_as_uint(static_cast<const float*>(p.C)[rb + e]);
-                                    }
-                                }
-                            }
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int r = r0 + i;
-                                const uint32_t srow = sbuf + (uint32_t)r * 128u;
-#pragma unroll
-                                for (int h = 0; h < EPR; ++h) {
-                                    const int e = (int)lane + 32 * h;
-                                    if constexpr (OUT == OUT_BF16)
-                                        st_shared_u16(srow + ((uint32_t)((e >> 3) ^ (r & 7)) << 4) + (uint32_t)(e & 7) * 2u,
-                                                      (uint16_t)x[i * EPR + h]);
-                                    else
-                                        st_shared_u32(srow + ((uint32_t)((e >> 2) ^ (r & 7)) << 4) + (uint32_t)(e & 3) * 4u,
-                                                      x[i * EPR + h]);
-                                }
-                            }
-                        }
-                        __syncwarp();
-                        if (row_in) {
-                            const uint32_t srow = sbuf + lane * 128u;
-#pragma unroll
-                            for (int cc = 0; cc < 8; ++cc) {
-                                uint32_t x0, x1, x2, x3;
-                                ld_shared_v4(srow + ((uint32_t)(cc ^ (int)(lane & 7u)) << 4), x0, x1, x2, x3);
-                                const uint32_t xs[4] = {x0, x1, x2, x3};
-#pragma unroll
-                                for (int h = 0; h < 4; ++h) {
-                                    if constexpr (OUT == OUT_BF16) {
-                                        const int e = 8 * cc + 2 * h;
-                                        if (colc + e < p.N) v[e] = fmaf(p.beta, __uint_as_float(xs[h] << 16), v[e]);
-                                        if (colc + e + 1 < p.N)
-                                            v[e + 1] = fmaf(p.beta, __uint_as_float(xs[h] & 0xFFFF0000u), v[e + 1]);
-                                    } else {
-                                        const int e = 4 * cc + h;
-                                        if (colc + e < p.N) v[e] = fmaf(p.beta, __uint_as_float(xs[h]), v[e]);
-                                    }
-                                }
-                            }
-                        }
-                        __syncwarp();  // every lane has its C_in before the buffer is overwritten
-                    } else if (p.c_read && row_in) {
-                        if (full_cols && p.c_tma) {
-                            if constexpr (OUT == OUT_BF16) {
-                                const uint4* src = reinterpret_cast<const uint4*>(
-                                    static_cast<const uint16_t*>(p.C) + cbase + colc);
-#pragma unroll
-                                for (int j = 0; j < T::STG_COLS / 8; ++j) {
-                                    const uint4 w = src[j];
-                                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                                    for (int h = 0; h < 4; ++h) {
-                                        v[8 * j + 2 * h] =
-                                            fmaf(p.beta, __uint_as_float(ww[h] << 16), v[8 * j + 2 * h]);
-                                        v[8 * j + 2 * h + 1] = fmaf(
-                                            p.beta, __uint_as_float(ww[h] & 0xFFFF0000u), v[8 * j + 2 * h + 1]);
-                                    }
-                                }
-                            } else {
-                                const float4* src = reinterpret_cast<const float4*>(
-                                    static_cast<const float*>(p.C) + cbase + colc);
-#pragma unroll
-                                for (int j = 0; j < T::STG_COLS / 4; ++j) {
-                                    const float4 w = src[j];
-                                    v[4 * j + 0] = fmaf(p.beta, w.x, v[4 * j + 0]);
-                                    v[4 * j + 1] = fmaf(p.beta, w.y, v[4 * j + 1]);
-                                    v[4 * j + 2] = fmaf(p.beta, w.z, v[4 * j + 2]);
-                                    v[4 * j + 3] = fmaf(p.beta, w.w, v[4 * j + 3]);
-                                }
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < T::STG_COLS; ++j) {
-                                if (colc + j < p.N) {
-                                    float cin;
-                                    if constexpr (OUT == OUT_BF16)
-                                        cin = __uint_as_float(
-                                            (uint32_t)(static_cast<const uint16_t*>(p.C)[cbase + colc + j]) << 16);
-                                    else
-                                        cin = static_cast<const float*>(p.C)[cbase + colc + j];
-                                    v[j] = fmaf(p.beta, cin, v[j]);
-                                }
-                            }
-                        }
-                    }
-                    // pack the 128-byte row segment into 8 x 16-byte words
-                    uint32_t w[32];
-                    if constexpr (OUT == OUT_BF16) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                        finish_chunk(b, nb, row0, row, sub, c, v);
                     } else {
+                        // publish this slice's partial sums; the slot stays held for the fixup
+                        float* g = slab(sl) + (size_t)((sub * CPW + ci) * PIECES) * 1024;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
+                        for (int h = 0; h < PIECES; ++h) put_piece(g + h * 1024, v + 32 * h, stg + buf * T::STG_BYTES);
                     }
-                    if (ARES != 0 && p.c_tma && full_cols && row_in) {
-                        // whole 128-byte row segment of this thread, inside N: eight 16-byte stores
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<char*>(p.C) +
-                                                              (cbase + colc) * (OUT == OUT_BF16 ? 2 : 4));
+                }
+            }
+            if (S > 1 && ok) {
+                // Split-K fixup, per warp (its 32 rows).  Arrival is counted after the partial
+                // sums are visible; the last of the S slices to arrive adds them up in slice
+                // order 0..S-1, its own from TMEM, the others from global memory, so the result
+                // is the same whatever the arrival order.  Nothing waits on another CTA.
+                __threadfence();
+                __syncwarp();
+                unsigned int* cnt = p.counters + ((size_t)(t * CG + (int)rank) * T::EPI_WARPS + ew);
+                unsigned int old = 0;
+                if (lane == 0) {
+                    old = atomicAdd(cnt, 1u);
+                    if (old == (unsigned int)(S - 1)) *cnt = 0u;  // ready for the next call
+                }
+                old = __shfl_sync(0xffffffffu, old, 0);
+                if (old == (unsigned int)(S - 1)) {
+                    __threadfence();
+                    for (int sub = 0; sub < NSUB; ++sub) {
+                        const int slot = NSUB == 1 ? acc : sub;
+                        const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(slot * BN);
+#pragma unroll 1
+                        for (int ci = 0; ci < CPW; ++ci) {
+                            const int c = half * CPW + ci;
+                            float v[T::STG_COLS];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                    } else if (ARES == 0) {
-                        const uint32_t row_addr = sbuf + lane * 128u;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            st_shared_v4(row_addr + ((uint32_t)(j ^ (int)(lane & 7u)) << 4), w[4 * j],
-                                         w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                        if (tma_chunk) {
-                            fence_proxy_async_smem();
+                            for (int j = 0; j < T::STG_COLS; ++j) v[j] = 0.0f;
+                            const size_t off = (size_t)((sub * CPW + ci) * PIECES) * 1024;
+                            // the buffer finish_chunk will use next; a tensor store may still read it
+                            if (lane == 0) bulk_wait_group_read<T::STG_BUFS - 1>();
                             __syncwarp();
-                            if (lane == 0) {
-                                tma_store_3d(&tmC, sbuf, colc, row0, bb);
-                                bulk_commit_group();
-                            }
-                        } else {
-                            // row by row: lane j writes element j (and j+32) of each row, coalesced
-                            __syncwarp();
-#pragma unroll 8
-                            for (int r = 0; r < 32; ++r) {
-                                const int rr = row0 + r;
-                                if (rr >= p.M || bb >= p.batch_real) continue;
-                                const long long rb = (long long)bb * p.stride_c + (long long)rr * p.ldc + colc;
-                                const uint32_t srow = sbuf + (uint32_t)r * 128u;
-                                if constexpr (OUT == OUT_BF16) {
+                            const uint32_t sb = stg + buf * T::STG_BYTES;
+#pragma unroll 1
+                            for (int s2 = 0; s2 < S; ++s2) {
+                                if (s2 == sl) {
+                                    float own[T::STG_COLS];
+                                    load_chunk(trow, c, own);
 #pragma unroll
-                                    for (int h = 0; h < 2; ++h) {
-                                        const int e = (int)lane + 32 * h;
-                                        if (colc + e < p.N)
-                                            static_cast<uint16_t*>(p.C)[rb + e] = ld_shared_u16(
-                                                srow + ((uint32_t)((e >> 3) ^ (r & 7)) << 4) + (uint32_t)(e & 7) * 2u);
+                                    for (int j = 0; j < T::STG_COLS; ++j) v[j] += own[j];
+                                    continue;
+                                }
+                                // every piece of the chunk in flight at once, then through the buffer
+                                const uint4* g = reinterpret_cast<const uint4*>(slab(s2) + off);
+                                uint4 x[PIECES][8];
+#pragma unroll
+                                for (int h = 0; h < PIECES; ++h)
+#pragma unroll
+                                    for (int i = 0; i < 8; ++i) x[h][i] = __ldcg(g + h * 256 + i * 32 + (int)lane);
+#pragma unroll
+                                for (int h = 0; h < PIECES; ++h) {
+#pragma unroll
+                                    for (int i = 0; i < 8; ++i)
+                                        st_shared_v4(sb + (uint32_t)i * 512u + lane * 16u, x[h][i].x, x[h][i].y,
+                                                     x[h][i].z, x[h][i].w);
+                                    __syncwarp();
+#pragma unroll
+                                    for (int j = 0; j < 8; ++j) {
+                                        uint32_t y0, y1, y2, y3;
+                                        ld_shared_v4(sb + lane * 128u + ((uint32_t)(j ^ (int)(lane & 7u)) << 4), y0, y1,
+                                                     y2, y3);
+                                        v[32 * h + 4 * j] += __uint_as_float(y0);
+                                        v[32 * h + 4 * j + 1] += __uint_as_float(y1);
+                                        v[32 * h + 4 * j + 2] += __uint_as_float(y2);
+                                        v[32 * h + 4 * j + 3] += __uint_as_float(y3);
                                     }
-                                } else {
-                                    const int e = (int)lane;
-                                    if (colc + e < p.N)
-                                        static_cast<float*>(p.C)[rb + e] = __uint_as_float(ld_shared_u32(
-                                            srow + ((uint32_t)((e >> 2) ^ (r & 7)) << 4) + (uint32_t)(e & 3) * 4u));
+                                    __syncwarp();
                                 }
                             }
-                            __syncwarp();
-                        }
-                        if (T::STG_BUFS == 2) buf ^= 1;
-                    } else if (row_in) {
-                        if constexpr (OUT == OUT_BF16) {
-                            uint16_t* dst = static_cast<uint16_t*>(p.C) + cbase + colc;
-#pragma unroll
-                            for (int j = 0; j < T::STG_COLS; ++j)
-                                if (colc + j < p.N)
-                                    dst[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
-                        } else {
-                            float* dst = static_cast<float*>(p.C) + cbase + colc;
-#pragma unroll
-                            for (int j = 0; j < T::STG_COLS; ++j)
-                                if (colc + j < p.N) dst[j] = __uint_as_float(w[j]);
+                            finish_chunk(b, nb, row0, row, sub, c, v);
                         }
                     }
+                }
+            }
+            if (S > 1) {
+                // the unit's accumulator slots are free again
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (NSUB == 1) mbar_arrive_cluster(tempty_leader0 + 8u * acc);
+                    else
+                        for (int sub = 0; sub < NSUB; ++sub) mbar_arrive_cluster(tempty_leader0 + 8u * sub);
                 }
             }
             if (NSUB == 1) acc ^= 1;

@@ -15,10 +15,13 @@
  * All matrices are row-major in device memory; leading dimensions and strides are in
  * ELEMENTS.  Calls are asynchronous: they validate the arguments, enqueue the kernels on
  * `stream` and return.  The caller owns every buffer it passes; the library never frees
- * them.  The library owns only a stream-ordered workspace (taken from the device's default
- * memory pool with cudaMallocAsync and released with cudaFreeAsync on `stream`) that is
- * used when A or B cannot be read by the tensor-memory accelerator as given (a leading
- * dimension that is not a multiple of 8 elements, a base not 16-byte aligned).
+ * them.  The library owns only a stream-ordered workspace, taken on `stream` from a memory
+ * pool of its own (one per device, created on first use) and given back on `stream` at the end
+ * of the call.  It holds the padded copies of A or B when the tensor-memory accelerator cannot
+ * read them as given (a leading dimension that is not a multiple of 8 elements, a base not
+ * 16-byte aligned), and the fp32 partial sums when a call with few output tiles cuts K into
+ * slices (split-K).  The pool keeps freed memory for later calls rather than returning it to
+ * the driver, so it holds the largest workspace used so far until the process exits.
  *
  * No exceptions cross this boundary.  Nothing is enqueued when a call returns an error.
  */

@@ -194,6 +194,64 @@ def test_deterministic(pw, plan):
     assert torch.equal(C1, C2)
 
 
+# ----------------------------------------------------------------------------- split-K
+# (M, N, K, slices): every slice count divides the k-blocks (BK = 64) into equal runs but the
+# last, and the K tail (K % 64 != 0) lands in the last slice.
+SPLIT_CASES = [(300, 200, 1100, 2), (129, 257, 1500, 3), (1000, 136, 2000, 5), (256, 512, 1024, 8)]
+STREAM_PLANS = [0, 1, 2, 3, 4]
+
+
+@pytest.mark.parametrize("plan", STREAM_PLANS)
+@pytest.mark.parametrize("case", SPLIT_CASES, ids=[f"{m}x{n}x{k}_s{s}" for m, n, k, s in SPLIT_CASES])
+def test_split_k(pw, plan, case, monkeypatch):
+    """K cut into slices whose fp32 partial sums the last-arriving unit adds in slice order:
+    same tolerance as the unsplit path, C read in place with alpha/beta, ragged M and N."""
+    M, N, K, S = case
+    monkeypatch.setenv("GEMM_BF16_SPLIT_K", str(S))
+    _plan(pw, plan)
+    A = matrix_bf16(61, M, K)
+    B = matrix_bf16(62, N, K)
+    c0bits = matrix_bf16(63, M, N)
+    c0 = torch.from_numpy(bf16_bits_to_f64(c0bits)).to(torch.bfloat16)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16, alpha=0.5, beta=1.0, c0=c0)
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, c0=c0bits, alpha=0.5, beta=1.0)
+    rep = check(values_f64(C), Cref, R, out_bf16=True)
+    assert rep["ok"], rep
+    # the same call again gives the same bits whatever order the slices arrived in
+    C2, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16, alpha=0.5, beta=1.0, c0=c0)
+    assert torch.equal(C, C2)
+
+
+@pytest.mark.parametrize("plan", STREAM_PLANS)
+def test_split_k_integer_bit_exact(pw, plan, monkeypatch):
+    """Small-integer inputs: slice sums and their total are exact in fp32, so a split GEMM must
+    match the oracle bit for bit."""
+    monkeypatch.setenv("GEMM_BF16_SPLIT_K", "4")
+    _plan(pw, plan)
+    rng = np.random.default_rng(200 + plan)
+    M, N, K = 384, 272, 2048
+    A = f64_to_bf16_bits(rng.integers(-3, 4, (M, K)).astype(np.float64))
+    B = f64_to_bf16_bits(rng.integers(-3, 4, (N, K)).astype(np.float64))
+    Cref, _ = oracle.gemm(A, B, M=M, N=N, K=K)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.float32)
+    assert np.array_equal(values_f64(C), Cref)
+
+
+def test_split_k_unaligned_c(pw, monkeypatch):
+    """Split-K with an odd ldc: the fixup goes out through the row-by-row coalesced store."""
+    monkeypatch.setenv("GEMM_BF16_SPLIT_K", "2")
+    _plan(pw, -1)
+    M, N, K = 261, 133, 1203
+    A = matrix_bf16(71, M, K, ld=K)
+    B = matrix_bf16(72, N, K, ld=K + 2)
+    c0bits = matrix_bf16(73, M, N, ld=N)
+    c0 = torch.from_numpy(bf16_bits_to_f64(c0bits)).to(torch.bfloat16)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16, alpha=0.5, beta=1.0, c0=c0, ldc=N)
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, c0=c0bits, alpha=0.5, beta=1.0)
+    rep = check(values_f64(C), Cref, R, out_bf16=True)
+    assert rep["ok"], rep
+
+
 def test_abi_errors_on_gpu(pw):
     c = pw.capi
     t = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
