@@ -436,13 +436,15 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             if (p.c_read && coop_chunk) {
                 // C_in: lane j reads elements j (and j+32 for bf16) of each of the warp's 32
                 // rows; element e of row r sits in 16-byte chunk (e*ES/16) ^ (r & 7).  Rows
-                // go 8 at a time so that 8 (16 for bf16) loads per lane are in flight.
+                // go RB at a time so that RB (2 RB for bf16) loads per lane are in flight:
+                // 16 rows keep the register budget of the other paths (32 spill).
+                constexpr int RB = 16;
                 constexpr int EPR = OUT == OUT_BF16 ? 2 : 1;  // elements per lane and row
 #pragma unroll 1
-                for (int r0 = 0; r0 < 32; r0 += 8) {
-                    uint32_t x[8 * EPR];
+                for (int r0 = 0; r0 < 32; r0 += RB) {
+                    uint32_t x[RB * EPR];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
+                    for (int i = 0; i < RB; ++i) {
                         const int rr = row0 + r0 + i;
                         const bool rv = rr < p.M && bb < p.batch_real;
                         const long long rb = (long long)bb * p.stride_c + (long long)rr * p.ldc + colc;
@@ -459,7 +461,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                         }
                     }
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
+                    for (int i = 0; i < RB; ++i) {
                         const int r = r0 + i;
                         const uint32_t srow = sbuf + (uint32_t)r * 128u;
 #pragma unroll
