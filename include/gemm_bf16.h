@@ -124,6 +124,14 @@ GEMM_API gemm_status_t gemm_bf16_device_status(struct CUstream_st* stream);
  * multiple of 64 that divides the tile width.
  * Returns GEMM_ERR_INVALID_ARG for an unknown plan.  A plan that cannot serve a given
  * call is replaced by the automatic choice for that call.
+ *
+ * With few output tiles and a long K, plans 0-4 may also cut K into slices (split-K): each
+ * (tile, slice) unit writes fp32 partial sums to the workspace and the last unit of a tile
+ * adds them in slice order, so results stay bitwise reproducible.  The plan and the slice
+ * count come from a cost model; environment variables read at every call override it for
+ * sweeps and tests:
+ *   GEMM_BF16_SPLIT_K=s     (1..8) s slices wherever the plan and K allow it (1: never split)
+ *   GEMM_BF16_GROUP_M=g     (1..64) m-blocks per group of the persistent tile order
  */
 GEMM_API gemm_status_t gemm_bf16_set_plan(int plan);
 
