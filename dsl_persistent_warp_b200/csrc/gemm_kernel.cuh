@@ -69,7 +69,7 @@ struct KParams {
                              // u / splits and k-blocks [s*kb_per_split, (s+1)*kb_per_split), s = u % splits
     int kb_per_split;
     float* ws;               // split-K partials: per (tile, CTA rank, slice) the CTA's 128 rows x
-                             // TILE_N columns in fp32, column-major (element (r, c) at c*128 + r)
+                             // TILE_N columns in fp32, as 4 KiB pieces per epilogue warp
     unsigned int* counters;  // split-K arrivals per (tile, CTA rank, epilogue warp); zero on entry,
                              // and the last arrival puts it back to zero
     int test_stall;          // test hook: the producer issues nothing, so the first bounded

@@ -296,6 +296,36 @@ def test_batched_shared_w(pw, plan, case):
         assert rep["ok"], (out, rep)
 
 
+# (batch, M, N, K, slices): N = 128 and 64 are packed several entries to a wide tile by
+# plans 1, 2 and 4; the others take one entry per tile.
+SPLIT_BATCH_CASES = [(3, 256, 128, 1024, 2), (5, 100, 72, 1100, 3), (4, 128, 64, 2048, 4)]
+
+
+@pytest.mark.parametrize("plan", STREAM_PLANS)
+@pytest.mark.parametrize("case", SPLIT_BATCH_CASES,
+                         ids=[f"b{b}_{m}x{n}x{k}_s{s}" for b, m, n, k, s in SPLIT_BATCH_CASES])
+def test_batched_split_k(pw, plan, case, monkeypatch):
+    """Split-K on the batched shared-W call: tiles over (b, n) with MN-major X, packing included."""
+    batch, M, N, K, S = case
+    monkeypatch.setenv("GEMM_BF16_SPLIT_K", str(S))
+    _plan(pw, plan)
+    ldx = N + (8 - N % 8) % 8
+    W = matrix_bf16(81, M, K, std=K ** -0.5)
+    X = matrix_bf16(82, batch * K, N, ld=ldx)
+    dW = to_dev_bf16(W)
+    dX = to_dev_bf16(X).view(batch, K, ldx)[:, :, :N]
+    y0 = torch.randn(batch, M, N, dtype=torch.float32).to(torch.bfloat16)
+    Y = y0.clone().cuda()
+    pw.gemm_bf16_batched_shared_w(dW, dX, Y, alpha=0.5, beta=1.0)
+    torch.cuda.synchronize()
+    assert pw.device_status() == 0
+    Cref, R = oracle.gemm_batched(W, X, batch=batch, M=M, N=N, K=K, stride_x=K * ldx,
+                                  y0=y0.to(torch.float32).numpy().reshape(batch * M, N),
+                                  stride_y=M * N, alpha=0.5, beta=1.0)
+    rep = check(values_f64(Y), Cref, R, out_bf16=True)
+    assert rep["ok"], rep
+
+
 # ----------------------------------------------------------------------------- full configs
 def _full_case(pw, idx, M, N, K, *, std_a=1.0, std_b=1.0, alpha=1.0, beta=0.0, rows=None):
     _plan(pw, -1)
