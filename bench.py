@@ -273,6 +273,11 @@ def run_ours(args, w, wname):
                 for _ in range(args.steps):
                     step()
             torch.cuda.synchronize()
+            # One untimed launch first: a graph that holds the library's workspace allocations
+            # maps their memory on its first launch (measured: twice the steady-state step time
+            # for the padded 4099^3 case); the timed launch is the steady state.
+            graph.replay()
+            torch.cuda.synchronize()
         except Exception:
             graph = None
             torch.cuda.synchronize()
@@ -405,7 +410,8 @@ def run_ours(args, w, wname):
             "l2": "inputs larger than L2" if algorithmic_bytes(w) > L2_BYTES else
                   "inputs smaller than L2 (steps back to back; no flush)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "timing": "cuda-graph replay of the timed steps" if graph is not None else "eager, events per step",
+            "timing": "cuda-graph replay of the timed steps (after one untimed launch of the graph)"
+                      if graph is not None else "eager, events per step",
         },
         "pct_of_peak": {
             "of_measured_burst": round(100.0 * value / world / peak_t, 2),
