@@ -371,6 +371,22 @@ def test_edge_shapes(pw, shape):
     _full_case(pw, 3, M, N, K, alpha=0.5, beta=1.0, rows=rows)
 
 
+# Few output tiles and a long K: the planner cuts K into slices on its own here.
+DEEP_K = [(1024, 1024, 8192), (512, 512, 16384), (384, 1000, 8192)]
+
+
+@pytest.mark.parametrize("shape", DEEP_K, ids=[f"{m}x{n}x{k}" for m, n, k in DEEP_K])
+def test_deep_k_auto_split(pw, shape):
+    """Automatic plan and split-K choice on deep-K shapes, alpha/beta with C in place, against
+    the oracle on every row; a second call must give the same bits."""
+    M, N, K = shape
+    C, A, B = _full_case(pw, 7, M, N, K, std_a=K ** -0.5, alpha=0.5, beta=1.0)
+    c0bits = matrix_bf16(seed_for(7, "C"), M, N)
+    c0 = torch.from_numpy(c0bits.view(np.int16)).view(torch.bfloat16)
+    C2, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16, alpha=0.5, beta=1.0, c0=c0)
+    assert torch.equal(C, C2)
+
+
 def test_recsys_batched_config(pw):
     """Y[b] = W X[b], b < 2048, W 256x512 ~ N(0, 1/sqrt(512)), X[b] 512x128 ~ N(0,1), bf16 out.
     All batches on sampled rows, and 16 whole batches."""
