@@ -440,23 +440,29 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 // 16 rows keep the register budget of the other paths (32 spill).
                 constexpr int RB = 16;
                 constexpr int EPR = OUT == OUT_BF16 ? 2 : 1;  // elements per lane and row
+                constexpr int ES = OUT == OUT_BF16 ? 2 : 4;   // bytes per element
+                const int nrows = bb < p.batch_real ? min(32, p.M - row0) : 0;
+                const char* src = static_cast<const char*>(p.C) +
+                                  ((long long)bb * p.stride_c + (long long)row0 * p.ldc + colc + (int)lane) * ES;
+                const long long sstep = (long long)p.ldc * ES;
+                bool ev[EPR];
+#pragma unroll
+                for (int h = 0; h < EPR; ++h) ev[h] = colc + (int)lane + 32 * h < p.N;
 #pragma unroll 1
                 for (int r0 = 0; r0 < 32; r0 += RB) {
                     uint32_t x[RB * EPR];
 #pragma unroll
                     for (int i = 0; i < RB; ++i) {
-                        const int rr = row0 + r0 + i;
-                        const bool rv = rr < p.M && bb < p.batch_real;
-                        const long long rb = (long long)bb * p.stride_c + (long long)rr * p.ldc + colc;
+                        const bool rv = r0 + i < nrows;
+                        const char* rp = src + (long long)(r0 + i) * sstep;
 #pragma unroll
                         for (int h = 0; h < EPR; ++h) {
-                            const int e = (int)lane + 32 * h;
                             x[i * EPR + h] = 0u;
-                            if (rv && colc + e < p.N) {
+                            if (rv && ev[h]) {
                                 if constexpr (OUT == OUT_BF16)
-                                    x[i * EPR + h] = static_cast<const uint16_t*>(p.C)[rb + e];
+                                    x[i * EPR + h] = *reinterpret_cast<const uint16_t*>(rp + 64 * h);
                                 else
-                                    x[i * EPR + h] = __float_as_uint(static_cast<const float*>(p.C)[rb + e]);
+                                    x[i * EPR + h] = *reinterpret_cast<const uint32_t*>(rp);
                             }
                         }
                     }
@@ -573,27 +579,39 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                         bulk_commit_group();
                     }
                 } else {
-                    // row by row: lane j writes element j (and j+32) of each row, coalesced
+                    // row by row: lane j writes element j (and j+32) of each row, coalesced.
+                    // The column predicates and the swizzle-free part of the shared address are
+                    // fixed for the lane and the global pointer advances by ldc, so a row costs
+                    // one shared load and one store per element (the loop is issue-bound: one
+                    // warp per scheduler, nothing else to hide latency behind).
                     __syncwarp();
-#pragma unroll 8
-                    for (int r = 0; r < 32; ++r) {
-                        const int rr = row0 + r;
-                        if (rr >= p.M || bb >= p.batch_real) continue;
-                        const long long rb = (long long)bb * p.stride_c + (long long)rr * p.ldc + colc;
-                        const uint32_t srow = sbuf + (uint32_t)r * 128u;
-                        if constexpr (OUT == OUT_BF16) {
+                    constexpr int ES = OUT == OUT_BF16 ? 2 : 4;  // bytes per element
+                    constexpr int EPR = OUT == OUT_BF16 ? 2 : 1;  // elements per lane and row
+                    const int nrows = bb < p.batch_real ? min(32, p.M - row0) : 0;
+                    char* dst = static_cast<char*>(p.C) +
+                                ((long long)bb * p.stride_c + (long long)row0 * p.ldc + colc + (int)lane) * ES;
+                    const long long dstep = (long long)p.ldc * ES;
+                    bool ev[EPR];
+                    uint32_t ch[EPR];
+                    const uint32_t inb = OUT == OUT_BF16 ? (lane & 7u) * 2u : (lane & 3u) * 4u;
 #pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                const int e = (int)lane + 32 * h;
-                                if (colc + e < p.N)
-                                    static_cast<uint16_t*>(p.C)[rb + e] = ld_shared_u16(
-                                        srow + ((uint32_t)((e >> 3) ^ (r & 7)) << 4) + (uint32_t)(e & 7) * 2u);
-                            }
-                        } else {
-                            const int e = (int)lane;
-                            if (colc + e < p.N)
-                                static_cast<float*>(p.C)[rb + e] = __uint_as_float(ld_shared_u32(
-                                    srow + ((uint32_t)((e >> 2) ^ (r & 7)) << 4) + (uint32_t)(e & 3) * 4u));
+                    for (int h = 0; h < EPR; ++h) {
+                        const int e = (int)lane + 32 * h;
+                        ev[h] = colc + e < p.N;
+                        ch[h] = (uint32_t)(e * ES / 16);
+                    }
+#pragma unroll 8
+                    for (int r = 0; r < nrows; ++r, dst += dstep) {
+                        const uint32_t srow = sbuf + (uint32_t)r * 128u + inb;
+                        const uint32_t sw = (uint32_t)(r & 7);
+#pragma unroll
+                        for (int h = 0; h < EPR; ++h) {
+                            if (!ev[h]) continue;
+                            const uint32_t a = srow + ((ch[h] ^ sw) << 4);
+                            if constexpr (OUT == OUT_BF16)
+                                *reinterpret_cast<uint16_t*>(dst + 64 * h) = ld_shared_u16(a);
+                            else
+                                *reinterpret_cast<uint32_t*>(dst) = ld_shared_u32(a);
                         }
                     }
                     __syncwarp();
