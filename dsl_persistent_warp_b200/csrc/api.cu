@@ -118,18 +118,19 @@ struct Req {
 struct PlanDesc {
     int cg, bn, nsub, stages, bk;  // CTAs per tile, MMA N, N sub-tiles per tile, ring stages, K per stage
     int ares;                      // A resident in shared memory (needs M <= 128*cg, K <= 512)
+    double rate;                   // TFLOP/s with every SM busy (B200, 8192^3 bf16); 0: never auto
 };
-constexpr int kNumPlans = 8;
-constexpr int kNumStreamPlans = 5;  // plans 0..4 stream both operands
+constexpr int kNumPlans = 9;
 constexpr PlanDesc kPlans[kNumPlans] = {
-    {1, 128, 1, 6, 64, 0},  // 0: 128x128, one CTA
-    {1, 256, 1, 4, 64, 0},  // 1: 128x256, one CTA
-    {2, 256, 1, 6, 64, 0},  // 2: 256x256, 2-CTA cluster
-    {2, 128, 1, 8, 64, 0},  // 3: 256x128, 2-CTA cluster
-    {2, 256, 2, 4, 64, 0},  // 4: 256x512, 2-CTA cluster, two 256-column MMA sub-tiles
-    {2, 128, 1, 12, 64, 1},  // 5: 256x128, 2-CTA cluster, A resident (M <= 256, K <= 512)
-    {1, 128, 1, 6, 64, 1},   // 6: 128x128, one CTA, A resident (M <= 128, K <= 512)
-    {2, 256, 1, 6, 64, 1},   // 7: 256x256, 2-CTA cluster, A resident (M <= 256, K <= 512)
+    {1, 128, 1, 6, 64, 0, 880.0},   // 0: 128x128, one CTA
+    {1, 256, 1, 4, 64, 0, 1190.0},  // 1: 128x256, one CTA
+    {2, 256, 1, 6, 64, 0, 1250.0},  // 2: 256x256, 2-CTA cluster
+    {2, 128, 1, 8, 64, 0, 790.0},   // 3: 256x128, 2-CTA cluster
+    {2, 256, 2, 4, 64, 0, 1400.0},  // 4: 256x512, 2-CTA cluster, two 256-column MMA sub-tiles
+    {2, 128, 1, 12, 64, 1, 0.0},    // 5: 256x128, 2-CTA cluster, A resident (M <= 256, K <= 512)
+    {1, 128, 1, 6, 64, 1, 0.0},     // 6: 128x128, one CTA, A resident (M <= 128, K <= 512)
+    {2, 256, 1, 6, 64, 1, 0.0},     // 7: 256x256, 2-CTA cluster, A resident (M <= 256, K <= 512)
+    {1, 64, 1, 8, 64, 0, 590.0},    // 8: 128x64, one CTA (twice the tiles of plan 0 on thin shapes)
 };
 
 // Batch entries packed side by side into one tile by plan `pd` (1 = no packing): needs the
@@ -197,10 +198,9 @@ gemm_status_t encode_3d(CUtensorMap* m, const void* base, bool f32, uint64_t d0,
     return res == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_CUDA;
 }
 
-// Sustained rate of each plan with every SM busy (TFLOP/s measured on B200, 8192^3 bf16); only
-// the ratios matter.  The automatic choice minimises the modelled time of plan_time() below:
-// large tiles move fewer operand bytes per FLOP, small tiles quantise better on small grids.
-constexpr double kPlanRate[kNumStreamPlans] = {880.0, 1190.0, 1250.0, 790.0, 1400.0};
+// The automatic choice minimises the modelled time of plan_time() below over the streaming
+// plans (rate > 0): large tiles move fewer operand bytes per FLOP, small tiles quantise better
+// on small grids.
 
 // Split-K limits: at most kMaxSplits slices of K, each at least kMinSplitKBlocks k-blocks long
 // (the smem ring needs a few blocks to fill), and a split must beat the unsplit choice by 10%.
@@ -240,7 +240,7 @@ double plan_time(int i, const Req& r, int sms, int splits) {
     const long long slots = sms / pd.cg;
     const long long kb = cdiv(cdiv(r.K, pd.bk), splits);  // k-blocks per unit
     const double unit_k = (double)(kb * pd.bk);
-    const double compute = 2.0 * (double)(tm * tn) * unit_k / (kPlanRate[i] * 1e12 / (double)slots);
+    const double compute = 2.0 * (double)(tm * tn) * unit_k / (pd.rate * 1e12 / (double)slots);
     const double stream = (double)(tm + tn) * unit_k * 2.0 / (pd.cg * kCtaOperandBytesPerSec);
     double t = (double)cdiv(plan_tiles(pd, r) * splits, slots) * (compute > stream ? compute : stream);
     if (splits > 1) {
@@ -280,21 +280,22 @@ struct Choice {
 Choice choose(const Req& r, int sms, bool allow_split) {
     const int fs = allow_split ? forced_splits() : 1;
     const int forced = g_plan_override.load();
-    int lo = 0, hi = kNumStreamPlans - 1;
+    int only = -1;  // the one plan to consider, or -1 for every streaming plan
     if (forced >= 0 && plan_serves(forced, r)) {
         if (kPlans[forced].ares) return {forced, 1};
-        lo = hi = forced;
+        only = forced;
     } else if (r.b_mn && r.K <= 1024 && pack_factor(kPlans[2], r.b_mn, r.N) > 1) {
         // Shared-W batched shapes with short K are bound by streaming X and Y through HBM: the
         // 256x256 tile holding several batch entries side by side measured fastest (W re-reads
         // hit L2); the resident-W plans (5-7) stay available through gemm_bf16_set_plan.
-        lo = hi = 2;
+        only = 2;
     }
-    Choice best{lo, 1};
+    Choice best{only >= 0 ? only : 0, 1};
     double best_t = 0.0;
     bool have = false;
-    for (int i = lo; i <= hi; ++i) {
+    for (int i = 0; i < kNumPlans; ++i) {
         const PlanDesc& pd = kPlans[i];
+        if (only >= 0 ? i != only : pd.rate <= 0.0) continue;
         const long long kb = cdiv(r.K, pd.bk);
         if (fs > 0) {
             const int s = split_valid(pd, r, fs) ? fs : 1;
@@ -394,6 +395,7 @@ gemm_status_t launch_by_plan(int plan, bool b_mn, int out, const CUtensorMap& ma
         case 5: return launch_plan<2, 128, 1, 12, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
         case 6: return launch_plan<1, 128, 1, 6, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
         case 7: return launch_plan<2, 256, 1, 6, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 8: return launch_plan<1, 64, 1, 8, 64, 0>(b_mn, out, ma, mb, mc, p, dev, sms, st);
         default: return GEMM_ERR_INVALID_ARG;
     }
 }

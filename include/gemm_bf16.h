@@ -120,12 +120,13 @@ GEMM_API gemm_status_t gemm_bf16_device_status(struct CUstream_st* stream);
  *   5: 256x128 tile, 2-CTA cluster, A resident in shared memory (M <= 256, K <= 512)
  *   6: 128x128 tile, one CTA, A resident in shared memory (M <= 128, K <= 512)
  *   7: 256x256 tile, 2-CTA cluster, A resident in shared memory (M <= 256, K <= 512)
+ *   8: 128x64 tile, one CTA (thin problems: twice the tiles of plan 0)
  * In the batched call, a tile wider than N holds several batch entries side by side when N is a
  * multiple of 64 that divides the tile width.
  * Returns GEMM_ERR_INVALID_ARG for an unknown plan.  A plan that cannot serve a given
  * call is replaced by the automatic choice for that call.
  *
- * With few output tiles and a long K, plans 0-4 may also cut K into slices (split-K): each
+ * With few output tiles and a long K, plans 0-4 and 8 may also cut K into slices (split-K): each
  * (tile, slice) unit writes fp32 partial sums to the workspace and the last unit of a tile
  * adds them in slice order, so results stay bitwise reproducible.  The plan and the slice
  * count come from a cost model; environment variables read at every call override it for

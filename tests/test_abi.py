@@ -96,9 +96,9 @@ def test_batched_rejects_bad_arguments(capi, args):
 
 
 def test_set_plan_and_timeout(capi):
-    assert capi.gemm_bf16_set_plan(8) == capi.GEMM_ERR_INVALID_ARG
+    assert capi.gemm_bf16_set_plan(9) == capi.GEMM_ERR_INVALID_ARG
     assert capi.gemm_bf16_set_plan(-2) == capi.GEMM_ERR_INVALID_ARG
-    for p in (0, 1, 2, 3, 4, 5, 6, 7, -1):
+    for p in (0, 1, 2, 3, 4, 5, 6, 7, 8, -1):
         assert capi.gemm_bf16_set_plan(p) == capi.GEMM_OK
     assert capi.gemm_bf16_set_wait_timeout_ns(0) == capi.GEMM_OK
 

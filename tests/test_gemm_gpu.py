@@ -13,7 +13,7 @@ from synth import bf16_bits_to_f64, f64_to_bf16_bits, matrix_bf16, seed_for
 
 pytestmark = pytest.mark.gpu
 
-PLANS = [0, 1, 2, 3, 4, 5, 6, 7]
+PLANS = [0, 1, 2, 3, 4, 5, 6, 7, 8]
 
 
 @pytest.fixture(scope="module")
@@ -198,7 +198,7 @@ def test_deterministic(pw, plan):
 # (M, N, K, slices): every slice count divides the k-blocks (BK = 64) into equal runs but the
 # last, and the K tail (K % 64 != 0) lands in the last slice.
 SPLIT_CASES = [(300, 200, 1100, 2), (129, 257, 1500, 3), (1000, 136, 2000, 5), (256, 512, 1024, 8)]
-STREAM_PLANS = [0, 1, 2, 3, 4]
+STREAM_PLANS = [0, 1, 2, 3, 4, 8]
 
 
 @pytest.mark.parametrize("plan", STREAM_PLANS)
