@@ -214,6 +214,12 @@ constexpr double kCtaOperandBytesPerSec = 140e9;
 constexpr double kSplitFixedSec = 4e-6;
 constexpr double kSplitWriteBytesPerSec = 45e9;
 constexpr double kSplitReadBytesPerSec = 90e9;
+// Fixed cost of one launch that the waves do not cover: pipeline fill, the exposed epilogue of
+// the last tiles and teardown.  Fitted on B200 to single-wave shapes (2048^3, 8192x512x4096,
+// 8192x256x4096, 127x8191x2048), where 2-CTA tiles pay more (the leader waits for both CTAs'
+// loads) and plan 1 beats plan 2 by 13 % although their waves model equal.
+constexpr double kLaunchFixedSecOneCta = 3e-6;
+constexpr double kLaunchFixedSecCtaPair = 6e-6;
 // Split-K arrival counters per CTA and tile: one per epilogue warp.
 constexpr int kSplitCountersPerCta = 4;
 
@@ -232,8 +238,9 @@ long long plan_tiles(const PlanDesc& pd, const Req& r) {
 }
 
 // Modelled time (s) of streaming plan `i` with K cut into `splits` slices: waves of work units,
-// each bound by the plan's per-cluster tensor rate or by its CTAs' operand streaming, plus,
-// when split, each unit's partial-sum write and the last unit's read of the other slices.
+// each bound by the plan's per-cluster tensor rate or by its CTAs' operand streaming, a fixed
+// cost per launch, and, when split, each unit's partial-sum write and the last unit's read of
+// the other slices.
 double plan_time(int i, const Req& r, int sms, int splits) {
     const PlanDesc& pd = kPlans[i];
     const long long tm = 128LL * pd.cg, tn = (long long)pd.bn * pd.nsub;
@@ -242,7 +249,8 @@ double plan_time(int i, const Req& r, int sms, int splits) {
     const double unit_k = (double)(kb * pd.bk);
     const double compute = 2.0 * (double)(tm * tn) * unit_k / (pd.rate * 1e12 / (double)slots);
     const double stream = (double)(tm + tn) * unit_k * 2.0 / (pd.cg * kCtaOperandBytesPerSec);
-    double t = (double)cdiv(plan_tiles(pd, r) * splits, slots) * (compute > stream ? compute : stream);
+    double t = (double)cdiv(plan_tiles(pd, r) * splits, slots) * (compute > stream ? compute : stream) +
+               (pd.cg == 2 ? kLaunchFixedSecCtaPair : kLaunchFixedSecOneCta);
     if (splits > 1) {
         const double partial = 128.0 * (double)tn * 4.0;  // bytes per CTA and unit
         t += kSplitFixedSec + partial / kSplitWriteBytesPerSec + (splits - 1) * partial / kSplitReadBytesPerSec;
@@ -290,27 +298,28 @@ Choice choose(const Req& r, int sms, bool allow_split) {
         // hit L2); the resident-W plans (5-7) stay available through gemm_bf16_set_plan.
         only = 2;
     }
+    // Unsplit plans first; a split must then beat the best of them by 10 %.
     Choice best{only >= 0 ? only : 0, 1};
     double best_t = 0.0;
     bool have = false;
     for (int i = 0; i < kNumPlans; ++i) {
         const PlanDesc& pd = kPlans[i];
         if (only >= 0 ? i != only : pd.rate <= 0.0) continue;
-        const long long kb = cdiv(r.K, pd.bk);
-        if (fs > 0) {
-            const int s = split_valid(pd, r, fs) ? fs : 1;
-            const double t = plan_time(i, r, sms, s);
-            if (!have || t < best_t * 0.999) best = {i, s}, best_t = t, have = true;
-            continue;
-        }
-        long long smax = kb / kMinSplitKBlocks;
-        if (pd.ares || smax < 1 || !allow_split) smax = 1;
+        const int s = fs > 0 && split_valid(pd, r, fs) ? fs : 1;
+        const double t = plan_time(i, r, sms, s);
+        if (!have || t < best_t * 0.999) best = {i, s}, best_t = t, have = true;
+    }
+    if (fs > 0 || !allow_split) return best;
+    const double split_bar = best_t * 0.90;
+    for (int i = 0; i < kNumPlans; ++i) {
+        const PlanDesc& pd = kPlans[i];
+        if (only >= 0 ? i != only : pd.rate <= 0.0) continue;
+        long long smax = cdiv(r.K, pd.bk) / kMinSplitKBlocks;
         if (smax > kMaxSplits) smax = kMaxSplits;
-        for (int s = 1; s <= (int)smax; ++s) {
-            if (!split_valid(pd, r, s)) continue;
-            const double t = plan_time(i, r, sms, s);
-            const double margin = s == 1 ? 0.999 : 0.90;
-            if (!have || t < best_t * margin) best = {i, s}, best_t = t, have = true;
+        for (int sp = 2; sp <= (int)smax; ++sp) {
+            if (!split_valid(pd, r, sp)) continue;
+            const double t = plan_time(i, r, sms, sp);
+            if (t < split_bar && t < best_t * 0.999) best = {i, sp}, best_t = t;
         }
     }
     return best;
