@@ -127,9 +127,9 @@ constexpr PlanDesc kPlans[kNumPlans] = {
     {2, 256, 1, 6, 64, 0, 1250.0},  // 2: 256x256, 2-CTA cluster
     {2, 128, 1, 8, 64, 0, 790.0},   // 3: 256x128, 2-CTA cluster
     {2, 256, 2, 4, 64, 0, 1400.0},  // 4: 256x512, 2-CTA cluster, two 256-column MMA sub-tiles
-    {2, 128, 1, 12, 64, 1, 0.0},    // 5: 256x128, 2-CTA cluster, A resident (M <= 256, K <= 512)
-    {1, 128, 1, 6, 64, 1, 0.0},     // 6: 128x128, one CTA, A resident (M <= 128, K <= 512)
-    {2, 256, 1, 6, 64, 1, 0.0},     // 7: 256x256, 2-CTA cluster, A resident (M <= 256, K <= 512)
+    {2, 128, 1, 8, 64, 1, 0.0},     // 5: 256x128, 2-CTA cluster, A resident (M <= 256, K <= 512)
+    {1, 128, 1, 4, 64, 1, 0.0},     // 6: 128x128, one CTA, A resident (M <= 128, K <= 512)
+    {2, 256, 1, 4, 64, 1, 0.0},     // 7: 256x256, 2-CTA cluster, A resident (M <= 256, K <= 512)
     {1, 64, 1, 8, 64, 0, 590.0},    // 8: 128x64, one CTA (twice the tiles of plan 0 on thin shapes)
 };
 
@@ -293,9 +293,11 @@ Choice choose(const Req& r, int sms, bool allow_split) {
         if (kPlans[forced].ares) return {forced, 1};
         only = forced;
     } else if (r.b_mn && r.K <= 1024 && pack_factor(kPlans[2], r.b_mn, r.N) > 1) {
-        // Shared-W batched shapes with short K are bound by streaming X and Y through HBM: the
-        // 256x256 tile holding several batch entries side by side measured fastest (W re-reads
-        // hit L2); the resident-W plans (5-7) stay available through gemm_bf16_set_plan.
+        // Shared-W batched shapes with short K are bound by streaming X and Y through HBM: a
+        // 256x256 tile holding several batch entries side by side, with W resident in shared
+        // memory when it fits (read once per CTA instead of once per tile from L2), measured
+        // fastest (RecSys 2048 x (256x512 . 512x128): plan 7 81.7 us, plan 2 84.5 us).
+        if (plan_serves(7, r)) return {7, 1};
         only = 2;
     }
     // Unsplit plans first; a split must then beat the best of them by 10 %.
@@ -401,9 +403,9 @@ gemm_status_t launch_by_plan(int plan, bool b_mn, int out, const CUtensorMap& ma
         case 2: return launch_plan<2, 256, 1, 6, 64, 0>(b_mn, out, ma, mb, mc, p, dev, sms, st);
         case 3: return launch_plan<2, 128, 1, 8, 64, 0>(b_mn, out, ma, mb, mc, p, dev, sms, st);
         case 4: return launch_plan<2, 256, 2, 4, 64, 0>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 5: return launch_plan<2, 128, 1, 12, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 6: return launch_plan<1, 128, 1, 6, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
-        case 7: return launch_plan<2, 256, 1, 6, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 5: return launch_plan<2, 128, 1, 8, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 6: return launch_plan<1, 128, 1, 4, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
+        case 7: return launch_plan<2, 256, 1, 4, 64, 1>(b_mn, out, ma, mb, mc, p, dev, sms, st);
         case 8: return launch_plan<1, 64, 1, 8, 64, 0>(b_mn, out, ma, mb, mc, p, dev, sms, st);
         default: return GEMM_ERR_INVALID_ARG;
     }

@@ -113,9 +113,7 @@ struct Tile {
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + (ARES ? KB_RES : STAGES) * A_BYTES;
     static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
-    // With A resident the epilogue stores rows straight from registers (no staging), leaving
-    // the shared memory to the B ring.
-    static constexpr int STG_REGION = ARES ? 0 : EPI_WARPS * STG_BUFS * STG_BYTES;
+    static constexpr int STG_REGION = EPI_WARPS * STG_BUFS * STG_BYTES;
     static constexpr int OFF_BAR = OFF_STG + STG_REGION;
     static constexpr int NUM_BARS = 2 * STAGES + 5;  // full/empty ring, tfull/tempty slots, resident A
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -423,14 +421,12 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             // chunk's end; otherwise (unaligned ldc, a ragged right edge) the warp moves it
             // row by row through the staging buffer so that every access is coalesced.
             const bool tma_chunk =
-                ARES == 0 && p.c_tma && colc + T::STG_COLS <= p.n_store_tma && bb < p.batch_real;
-            const bool coop_chunk = ARES == 0 && !tma_chunk;
+                p.c_tma && colc + T::STG_COLS <= p.n_store_tma && bb < p.batch_real;
+            const bool coop_chunk = !tma_chunk;
             const uint32_t sbuf = stg + buf * T::STG_BYTES;
-            if (ARES == 0) {
-                // the buffer may still be read by an earlier tensor store
-                if (lane == 0) bulk_wait_group_read<T::STG_BUFS - 1>();
-                __syncwarp();
-            }
+            // the buffer may still be read by an earlier tensor store
+            if (lane == 0) bulk_wait_group_read<T::STG_BUFS - 1>();
+            __syncwarp();
 #pragma unroll
             for (int j = 0; j < T::STG_COLS; ++j) v[j] *= p.alpha;
             if (p.c_read && coop_chunk) {
@@ -558,14 +554,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
 #pragma unroll
                 for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
             }
-            if (ARES != 0 && p.c_tma && full_cols && row_in) {
-                // whole 128-byte row segment of this thread, inside N: eight 16-byte stores
-                uint4* dst = reinterpret_cast<uint4*>(static_cast<char*>(p.C) +
-                                                      (cbase + colc) * (OUT == OUT_BF16 ? 2 : 4));
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-            } else if (ARES == 0) {
+            {
                 const uint32_t row_addr = sbuf + lane * 128u;
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
@@ -617,19 +606,6 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     __syncwarp();
                 }
                 if (T::STG_BUFS == 2) buf ^= 1;
-            } else if (row_in) {
-                if constexpr (OUT == OUT_BF16) {
-                    uint16_t* dst = static_cast<uint16_t*>(p.C) + cbase + colc;
-#pragma unroll
-                    for (int j = 0; j < T::STG_COLS; ++j)
-                        if (colc + j < p.N)
-                            dst[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
-                } else {
-                    float* dst = static_cast<float*>(p.C) + cbase + colc;
-#pragma unroll
-                    for (int j = 0; j < T::STG_COLS; ++j)
-                        if (colc + j < p.N) dst[j] = __uint_as_float(w[j]);
-                }
             }
         };
         // TMEM -> registers: chunk c (STG_COLS columns) of the slot whose lane-quarter row is trow.
