@@ -2,7 +2,7 @@
 rows, and the element-wise tolerance checks.
 
 Tolerances (float64 oracle values Cref, magnitude bound R = |alpha| sum|a||b| + |beta||c0|):
-  fp32 output:  |C - Cref| <= 1e-3 * R + 1e-5                     (as the task states it)
+  fp32 output:  |C - Cref| <= 1e-3 * R + 1e-5                     (the stated fp32 bound)
   bf16 output:  |C - Cref| <= 8e-3 * |Cref| + 1e-3 * R + 1e-5      (per element) and
                 ||C - Cref||_F <= 8e-3 * ||Cref||_F                (normwise)
 The stated "relative error <= 8e-3" for bf16 output is ill-posed where Cref ~ 0, so the
