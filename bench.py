@@ -536,12 +536,71 @@ def run_reference(args, w, wname):
     print(json.dumps(res), flush=True)
 
 
+def run_vendor(args, w, wname):
+    """Vendor context: the same workload through torch.matmul / addmm (cuBLAS), timed with the
+    same protocol as ours (W eager warm-up steps, K steps captured in a CUDA graph, one untimed
+    launch of the graph, one timed replay).  Rank 0 only; not a target and not part of the
+    product path."""
+    import torch
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    desc, batch, M, N, K, out, alpha, beta, *_ = w
+    base = {"metric": METRIC, "unit": UNIT, "impl": "vendor (torch.matmul, cuBLAS)",
+            "config": {"workload": desc, "name": wname}}
+    if out != "bf16":
+        # cuBLAS through torch has no bf16-in / fp32-out GEMM without converting the operands
+        print(json.dumps({**base, "unavailable": "fp32 output from bf16 operands"}), flush=True)
+        return
+    torch.cuda.set_device(0)
+    dA, dB, dC, _ = make_inputs(w, torch)
+
+    def step():
+        if batch > 1:
+            torch.matmul(dA, dB, out=dC)
+        elif beta != 0.0:
+            dC.addmm_(dA, dB.t(), beta=beta, alpha=alpha)
+        elif alpha != 1.0:
+            torch.mm(dA, dB.t(), out=dC).mul_(alpha)
+        else:
+            torch.mm(dA, dB.t(), out=dC)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(args.steps):
+            step()
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(0)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    sampler.start()
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    flops = 2.0 * batch * M * N * K
+    res = {**base, "value": round(flops * args.steps / (ms * 1e-3) / 1e12, 2), "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+           "higher_is_better": True, "dtype": "bf16", "data": "synthetic", "clocks": clocks}
+    del graph
+    print(json.dumps(res), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--impl", choices=["ours", "reference", "vendor"], default="ours",
+                    help="ours: this library; reference: the CPU oracle; vendor: torch.matmul (cuBLAS)")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=sorted(WORKLOADS) + ["all"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -557,6 +616,8 @@ def main():
     for n in names:
         if args.impl == "reference":
             run_reference(args, WORKLOADS[n], n)
+        elif args.impl == "vendor":
+            run_vendor(args, WORKLOADS[n], n)
         else:
             run_ours(args, WORKLOADS[n], n)
 
