@@ -23,7 +23,10 @@
  * slices (split-K).  The pool keeps freed memory for later calls rather than returning it to
  * the driver, so it holds the largest workspace used so far until the process exits.
  *
- * No exceptions cross this boundary.  Nothing is enqueued when a call returns an error.
+ * No exceptions cross this boundary.  A call rejected for its arguments enqueues nothing; a
+ * CUDA failure during the enqueue (GEMM_ERR_CUDA / GEMM_ERR_NO_MEMORY) may leave the steps
+ * already enqueued by that call on `stream` (pre-pass copies, the workspace's allocation and
+ * release), which touch only the workspace.
  */
 #ifndef GEMM_BF16_H
 #define GEMM_BF16_H
