@@ -49,10 +49,12 @@ def _lib(plant: int = 0, out_dir: str | None = None) -> ctypes.CDLL:
             LL = ctypes.c_longlong
             I = ctypes.c_int
             D = ctypes.c_double
-            lib.oracle_gemm.argtypes = [I, I, I, P, LL, P, LL, I, P, LL, I, D, D, P, I, P, P]
+            lib.oracle_gemm.argtypes = [I, I, I, P, LL, P, LL, I, P, LL, I, D, D, P, I, P, P, I]
             lib.oracle_gemm.restype = I
             lib.oracle_gemm_batched.argtypes = [I, I, I, I, P, LL, P, LL, LL, P, LL, LL, I, D,
-                                                D, P, I, P, P]
+                                                D, P, I, P, P, I]
+            lib.oracle_decode.argtypes = [I, P, LL, P]
+            lib.oracle_decode.restype = None
             lib.oracle_gemm_batched.restype = I
             lib.oracle_threads.restype = I
             lib.oracle_plant.restype = I
@@ -76,22 +78,51 @@ def _c0_type(c0: np.ndarray | None) -> int:
         return 1
     if c0.dtype == np.uint16:
         return 2
-    raise TypeError("c0 must be float32 or uint16 (bfloat16 bits)")
+    if c0.dtype == np.float16:
+        return 3
+    raise TypeError("c0 must be float32, uint16 (bfloat16 bits) or float16")
+
+
+_IN_TYPES = {"bf16": 0, "f16": 1}
+
+
+def _in_type(A: np.ndarray, in_dtype: str | None) -> int:
+    """16-bit operand type: explicit ``in_dtype`` ('bf16' / 'f16'), else fp16 for float16
+    arrays and bf16 for uint16 bit patterns."""
+    if in_dtype is not None:
+        return _IN_TYPES[in_dtype]
+    return 1 if A.dtype == np.float16 else 0
+
+
+def _bits(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float16:
+        return a.view(np.uint16)
+    return np.ascontiguousarray(a, dtype=np.uint16)
+
+
+def decode(h: np.ndarray, in_dtype: str, plant: int = 0, lib_dir: str | None = None) -> np.ndarray:
+    """Exact float64 values of 16-bit patterns ('bf16' or 'f16'), decoded by the oracle."""
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.empty(h.shape, dtype=np.float64)
+    _lib(plant, lib_dir).oracle_decode(_IN_TYPES[in_dtype], _ptr(h), int(h.size), _ptr(out))
+    return out
 
 
 def gemm(A: np.ndarray, B: np.ndarray, *, M: int, N: int, K: int, b_kmajor: bool = True,
          c0: np.ndarray | None = None, alpha: float = 1.0, beta: float = 0.0,
-         rows=None, plant: int = 0, lib_dir: str | None = None):
+         rows=None, plant: int = 0, lib_dir: str | None = None, in_dtype: str | None = None):
     """Reference rows of C = alpha*A*B + beta*c0.
 
-    A: uint16 (bf16 bits) 2-D, M x lda with lda >= K.
-    B: uint16 2-D; N x ldb (K-major, ``b_kmajor``) or K x ldb (N-major).
-    c0: None, or float32 / uint16 2-D M x ldc.
+    A: 2-D, M x lda with lda >= K: uint16 bit patterns (bf16 unless ``in_dtype`` = 'f16') or
+       float16.  B: the same type, 2-D; N x ldb (K-major, ``b_kmajor``) or K x ldb (N-major).
+    c0: None, or float32 / uint16 (bf16 bits) / float16 2-D M x ldc.
     rows: None (all M rows) or a sequence of row indices.
     Returns (Cref, R), float64 arrays of shape (len(rows), N).
     """
-    A = np.ascontiguousarray(A, dtype=np.uint16)
-    B = np.ascontiguousarray(B, dtype=np.uint16)
+    it = _in_type(A, in_dtype)
+    A = _bits(A)
+    B = _bits(B)
     lda = A.shape[1] if A.ndim == 2 and A.size else max(K, 1)
     ldb = B.shape[1] if B.ndim == 2 and B.size else max(K if b_kmajor else N, 1)
     if M and K:
@@ -114,7 +145,7 @@ def gemm(A: np.ndarray, B: np.ndarray, *, M: int, N: int, K: int, b_kmajor: bool
     R = np.empty((nrows, N), dtype=np.float64)
     rc = _lib(plant, lib_dir).oracle_gemm(
         M, N, K, _ptr(A), lda, _ptr(B), ldb, 1 if b_kmajor else 0, _ptr(c0), ldc,
-        _c0_type(c0), float(alpha), float(beta), _ptr(rows_arr), nrows, _ptr(Cref), _ptr(R))
+        _c0_type(c0), float(alpha), float(beta), _ptr(rows_arr), nrows, _ptr(Cref), _ptr(R), it)
     if rc != 0:
         raise ValueError("oracle_gemm rejected its arguments")
     return Cref, R
@@ -123,16 +154,19 @@ def gemm(A: np.ndarray, B: np.ndarray, *, M: int, N: int, K: int, b_kmajor: bool
 def gemm_batched(W: np.ndarray, X: np.ndarray, *, batch: int, M: int, N: int, K: int,
                  stride_x: int, y0: np.ndarray | None = None, stride_y: int = 0,
                  alpha: float = 1.0, beta: float = 0.0, rows=None, plant: int = 0,
-                 lib_dir: str | None = None):
+                 lib_dir: str | None = None, in_dtype: str | None = None):
     """Reference of Y[b] = alpha*W*X[b] + beta*Y0[b] for every b < batch.
 
-    W: uint16 2-D M x ldw.  X: uint16 1-D or 2-D buffer; X[b] starts at element b*stride_x
+    W: 2-D M x ldw, uint16 bit patterns (bf16 unless ``in_dtype`` = 'f16') or float16.
+    X: the same type, 1-D or 2-D buffer; X[b] starts at element b*stride_x
     and is K x N row-major with ldx = X.shape[-1] when 2-D (pass 2-D as (batch*K, ldx) or
-    (batch*K_pad, ldx)).  y0: None or float32/uint16 buffer laid out like Y, 2-D (rows, ldy).
+    (batch*K_pad, ldx)).  y0: None or float32/uint16/float16 buffer laid out like Y, 2-D
+    (rows, ldy).
     Returns (Cref, R) of shape (batch, len(rows), N).
     """
-    W = np.ascontiguousarray(W, dtype=np.uint16)
-    X = np.ascontiguousarray(X, dtype=np.uint16)
+    it = _in_type(W, in_dtype)
+    W = _bits(W)
+    X = _bits(X)
     ldw = W.shape[1]
     ldx = X.shape[-1]
     ldy = 0
@@ -150,7 +184,7 @@ def gemm_batched(W: np.ndarray, X: np.ndarray, *, batch: int, M: int, N: int, K:
     rc = _lib(plant, lib_dir).oracle_gemm_batched(
         batch, M, N, K, _ptr(W), ldw, _ptr(X), ldx, int(stride_x), _ptr(y0), ldy,
         int(stride_y), _c0_type(y0), float(alpha), float(beta), _ptr(rows_arr), nrows,
-        _ptr(Cref), _ptr(R))
+        _ptr(Cref), _ptr(R), it)
     if rc != 0:
         raise ValueError("oracle_gemm_batched rejected its arguments")
     return Cref, R

@@ -14,6 +14,9 @@ Definitions (all in numpy, vectorised, chunked to bound host memory):
 * ``f64_to_bf16_bits`` -- round-to-nearest-even from the float64 value straight to
   bfloat16 (8 significant bits), returned as uint16 bit patterns.  No double rounding
   through float32.
+* ``f64_to_f16_bits`` -- round-to-nearest-even from the float64 value straight to IEEE
+  binary16 (11 significant bits for normal values; a fixed quantum of 2^-24 below 2^-14,
+  the subnormal range), returned as uint16 bit patterns.
 
 Seeds: base 20261202; matrix ``role`` r in {A:0, B:1, C:2} of workload ``index`` i uses
 ``seed = base + 16*i + r``.
@@ -93,6 +96,36 @@ def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
 
 
+def f64_to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to IEEE binary16 (nearest, ties to even); uint16 bit patterns.
+
+    Finite inputs whose rounded magnitude stays at most 65504 (the largest fp16) only.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    if not np.all(np.isfinite(x)):
+        raise ValueError("non-finite value")
+    ax = np.abs(x)
+    normal = ax >= 2.0 ** -14
+    y = np.empty_like(x)
+    # normal range: float64 keeps 52 fraction bits, fp16 keeps 10: drop 42, round half even
+    bits = x[normal].view(np.uint64)
+    lsb = (bits >> np.uint64(42)) & np.uint64(1)
+    with np.errstate(over="ignore"):
+        rounded = (bits + np.uint64((1 << 41) - 1) + lsb) & ~np.uint64((1 << 42) - 1)
+    y[normal] = rounded.view(np.float64)
+    # subnormal range: multiples of 2^-24; scaling by 2^24 is exact and rint rounds half even
+    y[~normal] = np.rint(x[~normal] * 2.0 ** 24) * 2.0 ** -24
+    if np.any(np.abs(y) > 65504.0):
+        raise ValueError("value overflows fp16")
+    # every y is now an fp16 value, so this conversion is exact
+    return y.astype(np.float16).view(np.uint16)
+
+
+def f16_bits_to_f64(h: np.ndarray) -> np.ndarray:
+    """Exact float64 value of fp16 bit patterns."""
+    return np.ascontiguousarray(h, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
 def bf16_bits_to_f64(h: np.ndarray) -> np.ndarray:
     """Exact float64 value of bfloat16 bit patterns."""
     h = np.ascontiguousarray(h, dtype=np.uint16)
@@ -100,18 +133,23 @@ def bf16_bits_to_f64(h: np.ndarray) -> np.ndarray:
 
 
 def matrix_bf16(seed: int, rows: int, cols: int, dist: str = "normal", std: float = 1.0,
-                ld: int | None = None) -> np.ndarray:
+                ld: int | None = None, dtype: str = "bf16") -> np.ndarray:
     """A rows x cols bfloat16 matrix (uint16 bits) drawn row-major from stream ``seed``.
 
     Element (r, c) is stream element r*cols + c, whatever ``ld``; with ``ld`` > cols the
     padding columns are filled with the bfloat16 NaN pattern 0x7FC1 so that a kernel that
     reads them shows up in the results.
     dist: 'normal' (mean 0, standard deviation ``std``) or 'uniform' (on [-1, 1]).
+    dtype: 'bf16' (default) or 'f16' -- the 16-bit format the values are rounded to (the
+    padding then holds the fp16 NaN pattern 0x7E01).
     """
     ld = cols if ld is None else ld
     if ld < cols:
         raise ValueError("ld < cols")
-    out = np.full((rows, ld), 0x7FC1, dtype=np.uint16)
+    if dtype not in ("bf16", "f16"):
+        raise ValueError(dtype)
+    to_bits = f64_to_bf16_bits if dtype == "bf16" else f64_to_f16_bits
+    out = np.full((rows, ld), 0x7FC1 if dtype == "bf16" else 0x7E01, dtype=np.uint16)
     flat_total = rows * cols
     flat = np.empty(flat_total, dtype=np.uint16)
     for s in range(0, flat_total, _CHUNK):
@@ -122,6 +160,12 @@ def matrix_bf16(seed: int, rows: int, cols: int, dist: str = "normal", std: floa
             v = 2.0 * uniform01_f64(seed, s, n) - 1.0
         else:
             raise ValueError(dist)
-        flat[s:s + n] = f64_to_bf16_bits(v)
+        flat[s:s + n] = to_bits(v)
     out[:, :cols] = flat.reshape(rows, cols)
     return out
+
+
+def matrix_f16(seed: int, rows: int, cols: int, dist: str = "normal", std: float = 1.0,
+               ld: int | None = None) -> np.ndarray:
+    """``matrix_bf16`` with the values rounded to fp16 instead (uint16 bit patterns)."""
+    return matrix_bf16(seed, rows, cols, dist=dist, std=std, ld=ld, dtype="f16")

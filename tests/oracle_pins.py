@@ -18,6 +18,10 @@ What pins what:
   rows          a row subset equals the same rows of the full result
   batched       the batched call equals the single GEMM on each batch slice, and
                 exact rationals on a tiny batch
+  f16_decode    every one of the 65536 fp16 bit patterns decodes to numpy's float16 value
+  f16_golden    a hand-worked fp16 example (10-bit fractions, subnormal, 4096, c0 in fp16)
+  f16_integer   integer fp16 inputs beyond bf16's exact range agree with an int64 product
+  f16_fraction  tiny random fp16 inputs agree with exact rational arithmetic
 """
 from __future__ import annotations
 
@@ -27,7 +31,8 @@ from fractions import Fraction
 import numpy as np
 
 import oracle
-from synth import bf16_bits_to_f64, f64_to_bf16_bits, matrix_bf16
+from synth import (bf16_bits_to_f64, f16_bits_to_f64, f64_to_bf16_bits, f64_to_f16_bits, matrix_bf16,
+                   matrix_f16)
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 U53 = 2.0 ** -53
@@ -261,8 +266,74 @@ def pin_batched(plant=0, lib_dir=None):
     return ok, "batched == per-slice and exact"
 
 
+def pin_f16_decode(plant=0, lib_dir=None):
+    h = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.decode(h, "f16", plant=plant, lib_dir=lib_dir)
+    want = h.view(np.float16).astype(np.float64)  # numpy's own binary16 conversion
+    nan = np.isnan(want)
+    ok = np.array_equal(np.isnan(got), nan) and np.array_equal(got[~nan], want[~nan])
+    # signed zeros keep their sign
+    ok = ok and np.array_equal(np.signbit(got[~nan]), np.signbit(want[~nan]))
+    return ok, "all fp16 patterns"
+
+
+def _f16(vals, shape):
+    return f64_to_f16_bits(np.asarray(vals, dtype=np.float64)).reshape(shape)
+
+
+def pin_f16_golden(plant=0, lib_dir=None):
+    d = _read_golden("gemm_hand_f16_1x2x3.txt")
+    M, N, K = int(d["M"][0]), int(d["N"][0]), int(d["K"][0])
+    A = _f16(d["A"], (M, K))
+    Bs = _f16(d["Bs"], (N, K))
+    # the fixture's values must be fp16 values as written (no rounding on the way in)
+    ok0 = (np.array_equal(f16_bits_to_f64(A).ravel(), d["A"])
+           and np.array_equal(f16_bits_to_f64(Bs).ravel(), d["Bs"]))
+    C0 = np.asarray(d["C0"], dtype=np.float16).reshape(M, N)
+    C, _ = oracle.gemm(A, Bs, M=M, N=N, K=K, c0=C0, alpha=d["alpha"][0], beta=d["beta"][0],
+                       plant=plant, lib_dir=lib_dir, in_dtype="f16")
+    ok = ok0 and np.array_equal(C, np.asarray(d["C"]).reshape(M, N))
+    return ok, f"fp16 hand example: {ok}"
+
+
+def pin_f16_integer(plant=0, lib_dir=None):
+    rng = np.random.default_rng(19)
+    M, N, K = 21, 18, 1024
+    Ai = rng.integers(-300, 301, (M, K))  # exact in fp16 (11 significant bits), not in bf16
+    Bi = rng.integers(-300, 301, (N, K))
+    A = _f16(Ai, (M, K))
+    Bs = _f16(Bi, (N, K))
+    C, R = oracle.gemm(A, Bs, M=M, N=N, K=K, plant=plant, lib_dir=lib_dir, in_dtype="f16")
+    exact = Ai.astype(np.int64) @ Bi.astype(np.int64).T
+    rexact = np.abs(Ai).astype(np.int64) @ np.abs(Bi).astype(np.int64).T
+    return np.array_equal(C, exact) and np.array_equal(R, rexact), "integer fp16 inputs"
+
+
+def pin_f16_fraction(plant=0, lib_dir=None):
+    rng = np.random.default_rng(23)
+    for trial in range(12):
+        M, N, K = (int(x) for x in rng.integers(1, 8, 3))
+        kmajor = bool(trial % 2)
+        A = matrix_f16(400 + trial, M, K, std=0.01 if trial % 3 == 0 else 1.0)  # subnormals too
+        B = matrix_f16(500 + trial, N, K) if kmajor else matrix_f16(500 + trial, K, N)
+        b_kn = f16_bits_to_f64(B).T if kmajor else f16_bits_to_f64(B)
+        alpha = float(rng.choice([1.0, -0.5, 2.0]))
+        beta = float(rng.choice([0.0, 1.0, -0.25]))
+        c0 = matrix_f16(600 + trial, M, N).view(np.float16)
+        C, R = oracle.gemm(A, B, M=M, N=N, K=K, b_kmajor=kmajor, c0=c0, alpha=alpha, beta=beta,
+                           plant=plant, lib_dir=lib_dir, in_dtype="f16")
+        ex, bd = _exact_gemm(f16_bits_to_f64(A), b_kn, c0.astype(np.float64), alpha, beta)
+        for i in range(M):
+            for j in range(N):
+                tol = Fraction(K + 2) * Fraction(U53) * bd[i][j]
+                if abs(Fraction(C[i, j]) - ex[i][j]) > tol or abs(Fraction(R[i, j]) - bd[i][j]) > tol:
+                    return False, f"trial {trial} ({M},{N},{K}) elem ({i},{j})"
+    return True, "fp16 exact rationals"
+
+
 PINS = [pin_golden, pin_identity, pin_permutation, pin_rank1, pin_integer, pin_fraction,
-        pin_alpha_beta, pin_symmetry, pin_layouts, pin_rows, pin_batched]
+        pin_alpha_beta, pin_symmetry, pin_layouts, pin_rows, pin_batched, pin_f16_decode,
+        pin_f16_golden, pin_f16_integer, pin_f16_fraction]
 PLANTS = {
     1: "last k term dropped",
     2: "wrong sign on the beta term",
@@ -272,4 +343,5 @@ PLANTS = {
     6: "column index off by one",
     7: "running sums rounded to float32",
     8: "first k term dropped",
+    9: "fp16 exponent bias off by one",
 }
