@@ -52,7 +52,7 @@ def _lib(plant: int = 0, out_dir: str | None = None) -> ctypes.CDLL:
             lib.oracle_gemm.argtypes = [I, I, I, P, LL, P, LL, I, P, LL, I, D, D, P, I, P, P, I]
             lib.oracle_gemm.restype = I
             lib.oracle_gemm_batched.argtypes = [I, I, I, I, P, LL, P, LL, LL, P, LL, LL, I, D,
-                                                D, P, I, P, P, I]
+                                                D, P, I, P, P, I, P, I]
             lib.oracle_decode.argtypes = [I, P, LL, P]
             lib.oracle_decode.restype = None
             lib.oracle_gemm_batched.restype = I
@@ -184,7 +184,43 @@ def gemm_batched(W: np.ndarray, X: np.ndarray, *, batch: int, M: int, N: int, K:
     rc = _lib(plant, lib_dir).oracle_gemm_batched(
         batch, M, N, K, _ptr(W), ldw, _ptr(X), ldx, int(stride_x), _ptr(y0), ldy,
         int(stride_y), _c0_type(y0), float(alpha), float(beta), _ptr(rows_arr), nrows,
-        _ptr(Cref), _ptr(R), it)
+        _ptr(Cref), _ptr(R), it, None, 0)
     if rc != 0:
         raise ValueError("oracle_gemm_batched rejected its arguments")
+    return Cref, R
+
+
+def gemm_batched_dedup(W: np.ndarray, X: np.ndarray, index, *, n_x: int, M: int, N: int, K: int,
+                       stride_x: int, y0: np.ndarray | None = None, stride_y: int = 0,
+                       alpha: float = 1.0, beta: float = 0.0, rows=None, plant: int = 0,
+                       lib_dir: str | None = None, in_dtype: str | None = None):
+    """Reference of Y[b] = alpha*W*X[index[b]] + beta*Y0[b] for every b < len(index): the
+    deduplicated shared-W form, where X holds only the n_x distinct entries (X[u] starts at
+    element u*stride_x, K x N row-major with ldx = X.shape[-1]) and item b uses entry index[b].
+    Returns (Cref, R) of shape (len(index), len(rows), N)."""
+    it = _in_type(W, in_dtype)
+    W = _bits(W)
+    X = _bits(X)
+    idx = np.ascontiguousarray(np.asarray(index, dtype=np.int32))
+    batch = int(idx.size)
+    ldw = W.shape[1]
+    ldx = X.shape[-1]
+    ldy = 0
+    if y0 is not None:
+        y0 = np.ascontiguousarray(y0)
+        ldy = y0.shape[-1]
+    if rows is None:
+        rows_arr = None
+        nrows = M
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+        nrows = int(rows_arr.size)
+    Cref = np.empty((batch, nrows, N), dtype=np.float64)
+    R = np.empty((batch, nrows, N), dtype=np.float64)
+    rc = _lib(plant, lib_dir).oracle_gemm_batched(
+        batch, M, N, K, _ptr(W), ldw, _ptr(X), ldx, int(stride_x), _ptr(y0), ldy,
+        int(stride_y), _c0_type(y0), float(alpha), float(beta), _ptr(rows_arr), nrows,
+        _ptr(Cref), _ptr(R), it, _ptr(idx), int(n_x))
+    if rc != 0:
+        raise ValueError("oracle_gemm_batched rejected its arguments (index out of range?)")
     return Cref, R

@@ -225,20 +225,35 @@ int oracle_gemm(int M, int N, int K, const uint16_t* A, long long lda, const uin
  * (ldx) and Y0[b] = Y0 + b*stride_y (ldy).  Only the rows listed in rows[0..nrows-1]
  * (all M when rows == NULL) of each batch are produced; output batch b occupies
  * Cref[b*nrows*N ...].  This is the single-GEMM definition applied to each b in turn.
+ *
+ * With index != NULL (the deduplicated form: the request holds only the distinct feature
+ * entries, page "Meta accelere un noyau GPU d'un facteur 4 avec TLX...", sections "Comment le
+ * chargement des donnees gene le calcul" and "Ce que signifie une acceleration d'un facteur
+ * quatre"), item b's operand is the distinct entry index[b]: X[b] = X + index[b]*stride_x,
+ * 0 <= index[b] < n_x.  Each item is still its own plain GEMM.
  */
 int oracle_gemm_batched(int batch, int M, int N, int K, const uint16_t* W, long long ldw,
                         const uint16_t* X, long long ldx, long long stride_x, const void* Y0,
                         long long ldy, long long stride_y, int y_type, double alpha,
                         double beta, const int* rows, int nrows, double* Cref, double* R,
-                        int in_type) {
+                        int in_type, const int* index, int n_x) {
     if (batch < 0) return -1;
     if (!rows && nrows != M) return -1;
     long long per = (long long)nrows * N;
     for (int b = 0; b < batch; ++b) {
+        long long xb = b;
+        if (index) {
+#if ORACLE_PLANT == 10 /* planted: the item's own position used instead of its distinct entry */
+            xb = b % (n_x > 0 ? n_x : 1);
+#else
+            xb = index[b];
+#endif
+            if (xb < 0 || xb >= n_x) return -1;
+        }
         const void* yb = 0;
         if (y_type == 1) yb = (const float*)Y0 + (long long)b * stride_y;
         if (y_type == 2 || y_type == 3) yb = (const uint16_t*)Y0 + (long long)b * stride_y;
-        int rc = oracle_gemm(M, N, K, W, ldw, X + (long long)b * stride_x, ldx, 0, yb, ldy,
+        int rc = oracle_gemm(M, N, K, W, ldw, X + xb * stride_x, ldx, 0, yb, ldy,
                              y_type, alpha, beta, rows, nrows, Cref + b * per,
                              R ? R + b * per : (double*)0, in_type);
         if (rc) return rc;

@@ -22,6 +22,9 @@ What pins what:
   f16_golden    a hand-worked fp16 example (10-bit fractions, subnormal, 4096, c0 in fp16)
   f16_integer   integer fp16 inputs beyond bf16's exact range agree with an int64 product
   f16_fraction  tiny random fp16 inputs agree with exact rational arithmetic
+  dedup         the deduplicated shared-W form (items share distinct entries by index) equals
+                exact rationals per item on a tiny case, gives identical rows to items that
+                share an entry, and equals the batched form on the explicitly expanded batch
 """
 from __future__ import annotations
 
@@ -331,9 +334,36 @@ def pin_f16_fraction(plant=0, lib_dir=None):
     return True, "fp16 exact rationals"
 
 
+def pin_dedup(plant=0, lib_dir=None):
+    n_x, M, N, K = 3, 4, 5, 7
+    index = [2, 0, 2, 1, 2, 0]  # six items over three distinct entries
+    W = matrix_bf16(71, M, K)
+    X = matrix_bf16(72, n_x * K, N)
+    y0 = matrix_bf16(73, len(index) * M, N)
+    C, _ = oracle.gemm_batched_dedup(W, X, index, n_x=n_x, M=M, N=N, K=K, stride_x=K * N, y0=y0,
+                                     stride_y=M * N, alpha=-0.5, beta=1.0, plant=plant, lib_dir=lib_dir)
+    ok = True
+    for b, u in enumerate(index):
+        ex, bd = _exact_gemm(bf16_bits_to_f64(W), bf16_bits_to_f64(X[u * K:(u + 1) * K]),
+                             bf16_bits_to_f64(y0[b * M:(b + 1) * M]), -0.5, 1.0)
+        for i in range(M):
+            for j in range(N):
+                if abs(Fraction(C[b, i, j]) - ex[i][j]) > (K + 2) * Fraction(U53) * bd[i][j]:
+                    ok = False
+    # items 0, 2 and 4 share entry 2: with beta = 0 their rows are identical
+    C0, _ = oracle.gemm_batched_dedup(W, X, index, n_x=n_x, M=M, N=N, K=K, stride_x=K * N,
+                                      plant=plant, lib_dir=lib_dir)
+    same = np.array_equal(C0[0], C0[2]) and np.array_equal(C0[0], C0[4]) and np.array_equal(C0[1], C0[5])
+    # the batched form on the expanded batch X[b] = X[index[b]]
+    Xe = np.concatenate([X[u * K:(u + 1) * K] for u in index])
+    Ce, _ = oracle.gemm_batched(W, Xe, batch=len(index), M=M, N=N, K=K, stride_x=K * N, plant=plant,
+                                lib_dir=lib_dir)
+    return ok and same and np.array_equal(C0, Ce), f"exact: {ok}, shared rows: {same}"
+
+
 PINS = [pin_golden, pin_identity, pin_permutation, pin_rank1, pin_integer, pin_fraction,
         pin_alpha_beta, pin_symmetry, pin_layouts, pin_rows, pin_batched, pin_f16_decode,
-        pin_f16_golden, pin_f16_integer, pin_f16_fraction]
+        pin_f16_golden, pin_f16_integer, pin_f16_fraction, pin_dedup]
 PLANTS = {
     1: "last k term dropped",
     2: "wrong sign on the beta term",
@@ -344,4 +374,5 @@ PLANTS = {
     7: "running sums rounded to float32",
     8: "first k term dropped",
     9: "fp16 exponent bias off by one",
+    10: "dedup: item position used instead of its distinct entry",
 }
