@@ -5,10 +5,16 @@
                     [--workload square8192|square4096|llm_up|llm_down|edge4099|edge8192x256|
                                 edge127x8191|recsys|square256|all]
 
-A step is one GEMM (one launch of the persistent kernel) over the workload's synthetic
-inputs, already resident in HBM.  Timing: W untimed warm-up steps, then K steps between
-CUDA events on the launching stream, bracketed by a barrier and a device synchronize; the
-time is the max over ranks.  Multi-GPU runs are independent replicas (the GEMM needs no
+A step is one GEMM (one call: the persistent kernel, plus the alignment pre-pass copies when
+an operand needs them) over the workload's synthetic inputs, already resident in HBM.
+Timing: W untimed warm-up steps; the step is captured into a CUDA graph, and each of the K
+timed steps is one replay between two CUDA events on the launching stream.  Workloads whose
+data are smaller than twice the L2 cache get a 256 MiB write between steps (L2 flushed: cold
+cache), outside the events; larger ones run back to back.  The K steps are bracketed by a
+barrier and a device synchronize; the time is the max over ranks.  The line reports the mean
+(value, ms_per_step), median and minimum step time.  A separate sustained leg replays the
+step back to back for a few seconds (the part settles at its power cap) and is compared with
+the measured sustained peak.  Multi-GPU runs are independent replicas (the GEMM needs no
 exchange): value = total FLOPs of all ranks / max time.  `--impl reference` times the fp64
 CPU oracle (rank 0 only) on a bounded sample of the same workload.
 """
@@ -22,6 +28,7 @@ import statistics
 import sys
 import threading
 import time
+from typing import NamedTuple
 
 import numpy as np
 
@@ -33,8 +40,29 @@ UNIT = "TFLOP/s"
 SPEC_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 L2_BYTES = 126 * 2 ** 20
+FLUSH_BYTES = 256 * 2 ** 20
 
-# name -> (description, batch, M, N, K, out, alpha, beta, std_a, std_b, dist, config index)
+
+class Workload(NamedTuple):
+    desc: str
+    batch: int
+    M: int
+    N: int
+    K: int
+    out: str          # "f32", "bf16" or "f16"
+    alpha: float
+    beta: float
+    std_a: float
+    std_b: float
+    dist: str         # "normal" or "uniform"
+    idx: int          # configuration index (seeds)
+    in_dtype: str = "bf16"  # operand type: "bf16" or "f16"
+    n_unique: int = 0       # > 0: deduplicated batch, X holds this many distinct entries and
+                            # item b uses entry b * n_unique // batch (consecutive items share)
+
+
+# name -> Workload(description, batch, M, N, K, out, alpha, beta, std_a, std_b, dist, config
+# index[, operand type])
 WORKLOADS = {
     "square256": ("single GEMM M=N=K=256, U[-1,1], fp32 out", 1, 256, 256, 256, "f32", 1.0, 0.0,
                   1.0, 1.0, "uniform", 0),
@@ -54,7 +82,18 @@ WORKLOADS = {
                      127, 8191, 2048, "bf16", 0.5, 1.0, 1.0, 1.0, "normal", 3),
     "recsys": ("batched shared-W GEMM Y[b]=W X[b], b<2048, W 256x512 N(0,1/sqrt(512)), X[b] 512x128 "
                "N(0,1), bf16 out", 2048, 256, 128, 512, "bf16", 1.0, 0.0, 512 ** -0.5, 1.0, "normal", 4),
+    "recsys_dedup128": ("batched shared-W GEMM Y[b]=W X[index[b]], b<2048 as 16 requests of 128 items "
+                        "sharing one feature entry (16 distinct X entries), W 256x512, X 512x128, bf16 out",
+                        2048, 256, 128, 512, "bf16", 1.0, 0.0, 512 ** -0.5, 1.0, "normal", 4, "bf16", 16),
+    "recsys_dedup4": ("batched shared-W GEMM Y[b]=W X[index[b]], b<2048 with 4 items per distinct entry "
+                      "(512 distinct X entries), W 256x512, X 512x128, bf16 out",
+                      2048, 256, 128, 512, "bf16", 1.0, 0.0, 512 ** -0.5, 1.0, "normal", 4, "bf16", 512),
+    "square8192_f16": ("square GEMM M=N=K=8192, fp16 operands N(0,1), fp32 acc, fp16 out", 1, 8192, 8192,
+                       8192, "f16", 1.0, 0.0, 1.0, 1.0, "normal", 1, "f16"),
+    "square4096_f16": ("square GEMM M=N=K=4096, fp16 operands N(0,1), fp32 acc, fp16 out", 1, 4096, 4096,
+                       4096, "f16", 1.0, 0.0, 1.0, 1.0, "normal", 1, "f16"),
 }
+WORKLOADS = {k: Workload(*v) for k, v in WORKLOADS.items()}
 DEFAULT_WORKLOAD = "square8192"
 
 
@@ -96,16 +135,23 @@ def algorithmic_bytes(w) -> float:
     _, batch, M, N, K, out, alpha, beta, *_ = w
     es = 4 if out == "f32" else 2
     a = M * K * 2  # W / A read once
-    b = batch * N * K * 2
+    b = (w.n_unique or batch) * N * K * 2  # X: the distinct entries only when deduplicated
     c = batch * M * N * es * (2 if beta != 0.0 else 1)
-    return float(a + b + c)
+    idx = batch * 4 if w.n_unique else 0
+    return float(a + b + c + idx)
+
+
+def executed_flops(w) -> float:
+    """FLOPs the kernels execute: 2*M*N*K per distinct entry for a deduplicated batch, else per
+    item.  The reported TFLOP/s always count 2*M*N*K per item (the workload's logical work)."""
+    return 2.0 * (w.n_unique or w.batch) * w.M * w.N * w.K
 
 
 def launches_per_step(w) -> int:
     """Kernels of this library one call enqueues: the GEMM, plus one alignment pre-pass copy per
     operand whose leading dimension is not a multiple of 8 elements (packed ld here)."""
     _, batch, M, N, K, *_ = w
-    n = 1
+    n = 2 if w.n_unique else 1  # the deduplicated form also groups the items by entry
     if K % 8:
         n += 1  # A (lda = K)
     if (N if batch > 1 else K) % 8:
@@ -114,7 +160,8 @@ def launches_per_step(w) -> int:
 
 
 class ClockSampler(threading.Thread):
-    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs
+    (every 0.5 ms by default)."""
 
     REASONS = {
         "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
@@ -126,7 +173,7 @@ class ClockSampler(threading.Thread):
         "sync_boost": "nvmlClocksEventReasonSyncBoost",
     }
 
-    def __init__(self, torch_dev: int, period_s: float = 0.002):
+    def __init__(self, torch_dev: int, period_s: float = 0.0005):
         super().__init__(daemon=True)
         self.period = period_s
         self.samples = []
@@ -215,29 +262,62 @@ def aggregate_tflops(flops_per_step: float, steps: int, world: int, max_ms: floa
 def make_inputs(w, torch):
     """Seeded synthetic inputs on the device (packed leading dimensions)."""
     from synth import matrix_bf16, seed_for
-    desc, batch, M, N, K, out, alpha, beta, std_a, std_b, dist, idx = w
+    batch, M, N, K, idx = w.batch, w.M, w.N, w.K, w.idx
+    tdt = torch.float16 if w.in_dtype == "f16" else torch.bfloat16
 
-    def dev(bits, shape):
-        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).reshape(shape).cuda()
+    def draw(seed, rows, cols, std):
+        return matrix_bf16(seed, rows, cols, dist=w.dist, std=std, dtype=w.in_dtype)
+
+    def dev(bits, shape, dt=tdt):
+        return torch.from_numpy(bits.view(np.int16)).view(dt).reshape(shape).cuda()
 
     if batch == 1:
-        A = matrix_bf16(seed_for(idx, "A"), M, K, dist=dist, std=std_a)
-        B = matrix_bf16(seed_for(idx, "B"), N, K, dist=dist, std=std_b)
+        A = draw(seed_for(idx, "A"), M, K, w.std_a)
+        B = draw(seed_for(idx, "B"), N, K, w.std_b)
         dA, dB = dev(A, (M, K)), dev(B, (N, K))
-        host = {"A": A, "B": B}
     else:
-        A = matrix_bf16(seed_for(idx, "W"), M, K, dist=dist, std=std_a)
-        B = matrix_bf16(seed_for(idx, "X"), batch * K, N, dist=dist, std=std_b)
-        dA, dB = dev(A, (M, K)), dev(B, (batch, K, N))
-        host = {"A": A, "B": B}
-    odt = torch.float32 if out == "f32" else torch.bfloat16
+        nx = w.n_unique or batch
+        A = draw(seed_for(idx, "W"), M, K, w.std_a)
+        B = draw(seed_for(idx, "X"), nx * K, N, w.std_b)
+        dA, dB = dev(A, (M, K)), dev(B, (nx, K, N))
+    host = {"A": A, "B": B}
+    if w.n_unique:
+        host["index"] = dedup_index(w)
+    odt = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[w.out]
     shape = (M, N) if batch == 1 else (batch, M, N)
-    if beta != 0.0:
+    if w.beta != 0.0:
         Cb = matrix_bf16(seed_for(idx, "C"), batch * M, N)
-        dC = dev(Cb, shape).to(odt)
+        dC = dev(Cb, shape, torch.bfloat16).to(odt)
     else:
         dC = torch.empty(shape, dtype=odt, device="cuda")
     return dA, dB, dC, host
+
+
+def dedup_index(w) -> np.ndarray:
+    """Item b of a deduplicated workload uses distinct entry b * n_unique // batch."""
+    return (np.arange(w.batch, dtype=np.int64) * w.n_unique // w.batch).astype(np.int32)
+
+
+def needs_flush(w) -> bool:
+    """Data smaller than twice the L2 cache would stay cached from step to step: flush it."""
+    return algorithmic_bytes(w) < 2 * L2_BYTES
+
+
+def time_steps(torch, run_step, steps, stream, flush_buf=None):
+    """Device time (ms) of each of `steps` calls of run_step, each between two CUDA events on
+    `stream`; with `flush_buf`, a write of that buffer (larger than L2) precedes every step,
+    outside the events.  The host enqueues ahead of the device, so no host latency falls
+    between a step's events."""
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        if flush_buf is not None:
+            flush_buf.fill_(i & 0x7F)
+        starts[i].record(stream)
+        run_step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
 
 
 def run_ours(args, w, wname):
@@ -245,15 +325,18 @@ def run_ours(args, w, wname):
     import dsl_persistent_warp_b200 as pw
 
     world, rank, local = dist_setup(args.gpus)
-    desc, batch, M, N, K, out, alpha, beta, *_ = w
+    batch, M, N, K, out, alpha, beta = w.batch, w.M, w.N, w.K, w.out, w.alpha, w.beta
     flops = 2.0 * batch * M * N * K
     dA, dB, dC, host = make_inputs(w, torch)
+    dI = torch.from_numpy(host["index"]).cuda() if w.n_unique else None
 
-    def step(C=dC):
+    def step(A=dA, B=dB, C=dC, I=dI):
         if batch == 1:
-            pw.gemm_bf16(dA, dB, C, alpha=alpha, beta=beta)
+            pw.gemm_bf16(A, B, C, alpha=alpha, beta=beta)
+        elif w.n_unique:
+            pw.gemm_bf16_batched_shared_w_dedup(A, B, I, C, alpha=alpha, beta=beta)
         else:
-            pw.gemm_bf16_batched_shared_w(dA, dB, C, alpha=alpha, beta=beta)
+            pw.gemm_bf16_batched_shared_w(A, B, C, alpha=alpha, beta=beta)
 
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -262,61 +345,80 @@ def run_ours(args, w, wname):
     if pw.device_status() != 0:
         raise RuntimeError("kernel reported a bounded-wait timeout during warm-up")
 
-    # The K timed steps are captured once into a CUDA graph and replayed between two events, so
-    # the device time of small GEMMs is not hidden behind Python call overhead; if capture is
-    # not possible the steps run eagerly with an event pair around each one.
+    # Host cost of one call through the public API (Python wrapper, C ABI, planning, cached
+    # tensor maps, launch), measured on eager calls that the device runs back to back.
+    n_host = max(3, min(args.steps, 20))
+    t0 = time.perf_counter()
+    for _ in range(n_host):
+        step()
+    host_us = (time.perf_counter() - t0) * 1e6 / n_host
+    torch.cuda.synchronize()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if needs_flush(w) else None
+    eager_ms = time_steps(torch, step, n_host, stream, flush)
+
+    # The step captured once into a CUDA graph and replayed: the device time of small GEMMs is
+    # not hidden behind Python call overhead.  If capture is not possible the steps run eagerly.
     graph = None
     if not args.eager:
         try:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
-                for _ in range(args.steps):
-                    step()
+                step()
             torch.cuda.synchronize()
-            # One untimed launch first: a graph that holds the library's workspace allocations
-            # maps their memory on its first launch (measured: twice the steady-state step time
-            # for the padded 4099^3 case); the timed launch is the steady state.
-            graph.replay()
+            # Untimed launches first: a graph that holds the library's workspace allocations maps
+            # their memory on its first launch.
+            for _ in range(2):
+                graph.replay()
             torch.cuda.synchronize()
         except Exception:
             graph = None
             torch.cuda.synchronize()
+    run = graph.replay if graph is not None else step
     sampler = ClockSampler(local)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     sampler.start()
-    if graph is not None:
-        starts[0].record(stream)
-        graph.replay()
-        ends[-1].record(stream)
-    else:
-        for i in range(args.steps):
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
-    torch.cuda.synchronize()
+    step_ms = time_steps(torch, run, args.steps, stream, flush)
     barrier(world)
     clocks = sampler.stop()
-    total_ms = starts[0].elapsed_time(ends[-1])
-    if graph is not None:
-        avg_launch_ms = total_ms / args.steps  # back-to-back replay: the device never idles
-    else:
-        avg_launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
     if pw.device_status() != 0:
         raise RuntimeError("kernel reported a bounded-wait timeout in the timed region")
-    total_ms = max_over_ranks(total_ms, world)
+    total_ms = max_over_ranks(sum(step_ms), world)
     value = aggregate_tflops(flops, args.steps, world, total_ms)
+    avg_launch_ms = sum(step_ms) / args.steps
+
+    # Sustained leg: the same step back to back for a few seconds, so that the part reaches its
+    # power-capped steady state; compared with the measured sustained peak.
+    sustained = None
+    if args.sustained_seconds > 0 and world == 1:
+        n_sus = max(3, int(args.sustained_seconds / max(avg_launch_ms * 1e-3, 1e-6)))
+        sampler2 = ClockSampler(local, period_s=0.005)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        sampler2.start()
+        e0.record(stream)
+        for _ in range(n_sus):
+            run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        sus_clocks = sampler2.stop()
+        sus_ms = e0.elapsed_time(e1)
+        sustained = {"value": round(flops * n_sus / (sus_ms * 1e-3) / 1e12, 2), "unit": UNIT, "steps": n_sus,
+                     "seconds": round(sus_ms * 1e-3, 3), "clocks": sus_clocks,
+                     "l2": "back to back, no flush"}
+    used_graph = graph is not None
+    del graph
 
     # End to end through the public API with host buffers: every step copies its inputs from
     # pinned host memory, runs the GEMM and reads its result back, all inside the timed region.
     # Steps are pipelined over two device buffer sets and three streams (upload, compute,
     # download), so step i+1's upload overlaps step i's GEMM and step i-1's download.
-    hA = torch.from_numpy(host["A"].view(np.int16)).view(torch.bfloat16).reshape(dA.shape).pin_memory()
-    hB = torch.from_numpy(host["B"].view(np.int16)).view(torch.bfloat16).reshape(dB.shape).pin_memory()
+    hA = torch.from_numpy(host["A"].view(np.int16)).view(dA.dtype).reshape(dA.shape).pin_memory()
+    hB = torch.from_numpy(host["B"].view(np.int16)).view(dB.dtype).reshape(dB.shape).pin_memory()
     hC0 = dC.cpu().pin_memory() if beta != 0.0 else None
-    sets = [(dA, dB, dC), (torch.empty_like(dA), torch.empty_like(dB), torch.empty_like(dC))]
+    hI = torch.from_numpy(host["index"]).pin_memory() if w.n_unique else None
+    sets = [(dA, dB, dC, dI), (torch.empty_like(dA), torch.empty_like(dB), torch.empty_like(dC),
+                               torch.empty_like(dI) if dI is not None else None)]
     hCs = [torch.empty(dC.shape, dtype=dC.dtype).pin_memory() for _ in range(2)]
     s_up, s_mm, s_down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev_up = [torch.cuda.Event() for _ in range(2)]
@@ -327,7 +429,7 @@ def run_ours(args, w, wname):
     def e2e_run(n):
         for i in range(n):
             k = i % 2
-            a, bm, c = sets[k]
+            a, bm, c, ix = sets[k]
             with torch.cuda.stream(s_up):
                 if i >= 2:
                     s_up.wait_event(ev_mm[k])    # set k's inputs no longer read
@@ -336,15 +438,14 @@ def run_ours(args, w, wname):
                 bm.copy_(hB, non_blocking=True)
                 if hC0 is not None:
                     c.copy_(hC0, non_blocking=True)
+                if hI is not None:
+                    ix.copy_(hI, non_blocking=True)
                 ev_up[k].record(s_up)
             with torch.cuda.stream(s_mm):
                 s_mm.wait_event(ev_up[k])
                 if i >= 2:
                     s_mm.wait_event(ev_down[k])
-                if batch == 1:
-                    pw.gemm_bf16(a, bm, c, alpha=alpha, beta=beta)
-                else:
-                    pw.gemm_bf16_batched_shared_w(a, bm, c, alpha=alpha, beta=beta)
+                step(a, bm, c, ix)
                 ev_mm[k].record(s_mm)
             with torch.cuda.stream(s_down):
                 s_down.wait_event(ev_mm[k])
@@ -366,7 +467,8 @@ def run_ours(args, w, wname):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    h2d = hA.numel() * 2 + hB.numel() * 2 + (hC0.numel() * hC0.element_size() if hC0 is not None else 0)
+    h2d = (hA.numel() * 2 + hB.numel() * 2 + (hC0.numel() * hC0.element_size() if hC0 is not None else 0)
+           + (hI.numel() * 4 if hI is not None else 0))
     d2h = hCs[0].numel() * hCs[0].element_size()
     e2e_value = aggregate_tflops(flops, e2e_steps, world, e2e_ms)
     del sets
@@ -377,18 +479,21 @@ def run_ours(args, w, wname):
 
     peaks, peak_kind = load_peaks()
     peak_t = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_ts = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     peak_b = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     # Roofline of the step's dominant kernel: tensor-bound above the ridge point
-    # (peak FLOP/s / peak bytes/s), HBM-bound below it.
+    # (peak FLOP/s / peak bytes/s), HBM-bound below it.  fp16 and bf16 have the same dense
+    # tensor rate (kind::f16), so the bf16 peaks serve both.
     abytes = algorithmic_bytes(w)
-    hbm_bound = flops / abytes < peak_t * 1e12 / (peak_b * 1e9)
+    hbm_bound = executed_flops(w) / abytes < peak_t * 1e12 / (peak_b * 1e9)
     if hbm_bound:
         achieved, peak, r_unit = abytes / (avg_launch_ms * 1e-3) / 1e9, peak_b, "GB/s"
         peak_desc = f"HBM copy bandwidth ({peak_kind})"
     else:
-        achieved, peak, r_unit = flops / (avg_launch_ms * 1e-3) / 1e12, peak_t, "TFLOP/s"
-        peak_desc = f"bf16 dense, burst ({peak_kind})"
+        achieved, peak, r_unit = executed_flops(w) / (avg_launch_ms * 1e-3) / 1e12, peak_t, "TFLOP/s"
+        peak_desc = f"{w.in_dtype} dense, burst ({peak_kind}; the bf16 figure: same tensor rate)"
     traffic = recorded_traffic(wname)
+    flushed = flush is not None
     res = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -397,27 +502,30 @@ def run_ours(args, w, wname):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 5),
+        "median_ms": round(statistics.median(step_ms), 5),
+        "min_ms": round(min(step_ms), 5),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": w.in_dtype,
         "data": "synthetic",
         "config": {
-            "workload": desc,
+            "workload": w.desc,
             "name": wname,
             "batch": batch, "M": M, "N": N, "K": K,
-            "out": out, "alpha": alpha, "beta": beta,
-            "l2": "inputs larger than L2" if algorithmic_bytes(w) > L2_BYTES else
-                  "inputs smaller than L2 (steps back to back; no flush)",
+            "in": w.in_dtype, "out": out, "alpha": alpha, "beta": beta,
+            "l2": "flushed before every step (256 MiB write, outside the events)" if flushed else
+                  "inputs larger than L2 (steps back to back)",
+            "cold_l2": flushed,
+            **({"n_unique": w.n_unique, "flops": "counted per item (2*M*N*K per item), as for the "
+                "expanded batch; the distinct entries' GEMMs do batch/n_unique times fewer"}
+               if w.n_unique else {}),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "timing": "cuda-graph replay of the timed steps (after one untimed launch of the graph)"
-                      if graph is not None else "eager, events per step",
+            "timing": ("cuda-graph replay of one step, events around each replay"
+                       if used_graph else "eager, events around each step"),
         },
         "pct_of_peak": {
             "of_measured_burst": round(100.0 * value / world / peak_t, 2),
-            # cuBLAS looped for seconds under the 1000 W cap: the reference for long runs
-            "of_measured_sustained": round(100.0 * value / world / float(
-                peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])), 2),
             "of_spec_2250": round(100.0 * value / world / SPEC_BF16_TFLOPS, 2),
             "peak_source": peak_kind,
         },
@@ -431,12 +539,19 @@ def run_ours(args, w, wname):
             "algorithmic_bytes": abytes,
             "peak_kind": peak_desc,
         },
+        "eager": {"ms_per_step": round(statistics.mean(eager_ms), 5),
+                  "median_ms": round(statistics.median(eager_ms), 5),
+                  "host_us_per_call": round(host_us, 2), "calls": n_host},
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
                 "pipeline": "2 buffer sets; upload, GEMM and download on separate streams"},
         "gpu_launches": args.steps * launches_per_step(w),  # timed region of `value`
         "clocks": clocks,
     }
+    if sustained is not None:
+        sustained["frac_of_sustained_peak"] = round(sustained["value"] / peak_ts, 4)
+        sustained["sustained_peak"] = peak_ts
+        res["sustained"] = sustained
     if cpu is not None:
         res["cpu_baseline"] = cpu
     if rank == 0:
@@ -456,10 +571,15 @@ def cpu_baseline(w, host, budget_s=15.0):
         rows = list(range(nrows))
         t0 = time.perf_counter()
         if batch == 1:
-            oracle.gemm(A, B, M=M, N=N, K=K, rows=rows)
+            oracle.gemm(A, B, M=M, N=N, K=K, rows=rows, in_dtype=w.in_dtype)
+        elif w.n_unique:
+            nb = max(1, nrows // M)
+            oracle.gemm_batched_dedup(A, B, host["index"][:nb], n_x=w.n_unique, M=M, N=N, K=K,
+                                      stride_x=K * N, in_dtype=w.in_dtype)
         else:
             nb = max(1, nrows // M)
-            oracle.gemm_batched(A, B[: nb * K], batch=nb, M=M, N=N, K=K, stride_x=K * N)
+            oracle.gemm_batched(A, B[: nb * K], batch=nb, M=M, N=N, K=K, stride_x=K * N,
+                                in_dtype=w.in_dtype)
         return time.perf_counter() - t0
 
     if batch == 1:
@@ -486,25 +606,27 @@ def run_reference(args, w, wname):
         return
     import oracle
     from synth import matrix_bf16, seed_for
-    desc, batch, M, N, K, out, alpha, beta, std_a, std_b, dist, idx = w
+    desc, batch, M, N, K, out, alpha, beta, std_a, std_b, dist, idx = w[:12]
     # bounded sample: at most ~`ref_seconds` of CPU work over warmup + steps.
     total_steps = args.steps + args.warmup
     per_step_s = max(0.02, args.ref_seconds / max(total_steps, 1))
     # Rows of A are a prefix of its seeded stream, so only the rows a step can use are drawn.
     a_rows = min(M, 1024)
-    A = matrix_bf16(seed_for(idx, "A" if batch == 1 else "W"), a_rows, K, dist=dist, std=std_a)
+    A = matrix_bf16(seed_for(idx, "A" if batch == 1 else "W"), a_rows, K, dist=dist, std=std_a,
+                    dtype=w.in_dtype)
     if batch == 1:
-        B = matrix_bf16(seed_for(idx, "B"), N, K, dist=dist, std=std_b)
+        B = matrix_bf16(seed_for(idx, "B"), N, K, dist=dist, std=std_b, dtype=w.in_dtype)
     else:
-        B = matrix_bf16(seed_for(idx, "X"), K, N, dist=dist, std=std_b)
+        B = matrix_bf16(seed_for(idx, "X"), K, N, dist=dist, std=std_b, dtype=w.in_dtype)
     c0 = matrix_bf16(seed_for(idx, "C"), a_rows, N) if beta != 0.0 else None
 
     def one(nrows):
         rows = list(range(nrows))
         if batch == 1:
-            oracle.gemm(A, B, M=a_rows, N=N, K=K, c0=c0, alpha=alpha, beta=beta, rows=rows)
+            oracle.gemm(A, B, M=a_rows, N=N, K=K, c0=c0, alpha=alpha, beta=beta, rows=rows,
+                        in_dtype=w.in_dtype)
         else:
-            oracle.gemm(A, B, M=a_rows, N=N, K=K, b_kmajor=False, rows=rows)
+            oracle.gemm(A, B, M=a_rows, N=N, K=K, b_kmajor=False, rows=rows, in_dtype=w.in_dtype)
 
     t0 = time.perf_counter()
     one(1)
@@ -526,7 +648,8 @@ def run_reference(args, w, wname):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
         "config": {"workload": desc, "name": wname, "batch": batch, "M": M, "N": N, "K": K,
-                   "out": out, "alpha": alpha, "beta": beta, "parallelism": "host cores"},
+                   "in": w.in_dtype, "out": out, "alpha": alpha, "beta": beta,
+                   "parallelism": "host cores"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": oracle.threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -549,15 +672,20 @@ def run_vendor(args, w, wname):
     desc, batch, M, N, K, out, alpha, beta, *_ = w
     base = {"metric": METRIC, "unit": UNIT, "impl": "vendor (torch.matmul, cuBLAS)",
             "config": {"workload": desc, "name": wname}}
-    if out != "bf16":
-        # cuBLAS through torch has no bf16-in / fp32-out GEMM without converting the operands
-        print(json.dumps({**base, "unavailable": "fp32 output from bf16 operands"}), flush=True)
+    if out == "f32":
+        # cuBLAS through torch has no 16-bit-in / fp32-out GEMM without converting the operands
+        print(json.dumps({**base, "unavailable": "fp32 output from 16-bit operands"}), flush=True)
         return
     torch.cuda.set_device(0)
-    dA, dB, dC, _ = make_inputs(w, torch)
+    dA, dB, dC, host = make_inputs(w, torch)
+
+    dI = torch.from_numpy(host["index"]).long().cuda() if w.n_unique else None
 
     def step():
-        if batch > 1:
+        if w.n_unique:
+            # the distinct entries once, then each item's copy of its entry's result
+            torch.index_select(torch.matmul(dA, dB), 0, dI, out=dC)
+        elif batch > 1:
             torch.matmul(dA, dB, out=dC)
         elif beta != 0.0:
             dC.addmm_(dA, dB.t(), beta=beta, alpha=alpha)
@@ -589,7 +717,7 @@ def run_vendor(args, w, wname):
     flops = 2.0 * batch * M * N * K
     res = {**base, "value": round(flops * args.steps / (ms * 1e-3) / 1e12, 2), "n_gpus": 1,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
-           "higher_is_better": True, "dtype": "bf16", "data": "synthetic", "clocks": clocks}
+           "higher_is_better": True, "dtype": w.in_dtype, "data": "synthetic", "clocks": clocks}
     del graph
     print(json.dumps(res), flush=True)
 
@@ -609,11 +737,18 @@ def main():
                     help="CPU seconds for the whole --impl reference run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager calls instead of a graph replay")
+    ap.add_argument("--sustained-seconds", type=float, default=None,
+                    help="length of the back-to-back sustained leg (default: 3 s for tensor-bound "
+                         "workloads, 0 otherwise)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     names = sorted(WORKLOADS) if args.workload == "all" else [args.workload]
+    sustained_arg = args.sustained_seconds
     for n in names:
+        if sustained_arg is None:
+            w = WORKLOADS[n]
+            args.sustained_seconds = 3.0 if executed_flops(w) / algorithmic_bytes(w) > 263 else 0.0
         if args.impl == "reference":
             run_reference(args, WORKLOADS[n], n)
         elif args.impl == "vendor":

@@ -1,20 +1,26 @@
-"""Compile the CUDA library (csrc/*.cu -> libgemm_bf16.so, in-tree) for sm_100a with nvcc."""
+"""Compile the CUDA library (csrc/*.cu -> libgemm_bf16.so, in-tree) for sm_100a with nvcc.
+
+Each tile plan's kernels live in their own translation unit (csrc/plan*.cu), so the objects
+compile in parallel and are then linked into one shared library.
+"""
 from __future__ import annotations
 
 import glob
 import os
 import subprocess
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB_PATH = os.path.join(PKG, "libgemm_bf16.so")
-SOURCES = [os.path.join(PKG, "csrc", "api.cu")]
-DEPS = (glob.glob(os.path.join(PKG, "csrc", "*")) + [os.path.join(ROOT, "include", "gemm_bf16.h")])
+CSRC = os.path.join(PKG, "csrc")
+SOURCES = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+DEPS = (glob.glob(os.path.join(CSRC, "*")) + [os.path.join(ROOT, "include", "gemm_bf16.h")])
+OBJ_DIR = os.path.join(PKG, "_build")
 
-NVCC_FLAGS = [
-    "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
-    "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+NVCC_FLAGS = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler",
+              "-fvisibility=hidden"]
 
 
 def _nvcc() -> str:
@@ -29,15 +35,25 @@ def needs_build() -> bool:
     return any(os.path.getmtime(d) > t for d in DEPS if os.path.exists(d))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Build libgemm_bf16.so next to this file if it is missing or stale; return its path."""
-    if not force and not needs_build():
-        return LIB_PATH
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I" + os.path.join(ROOT, "include"), "-o", tmp, *SOURCES]
+def _compile(src: str, verbose: bool) -> str:
+    obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
+    cmd = [_nvcc(), *NVCC_FLAGS, "-I" + os.path.join(ROOT, "include"), "-c", "-o", obj, src]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
+    return obj
+
+
+def build(force: bool = False, verbose: bool = False, jobs: int | None = None) -> str:
+    """Build libgemm_bf16.so next to this file if it is missing or stale; return its path."""
+    if not force and not needs_build():
+        return LIB_PATH
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    jobs = jobs or max(1, min(len(SOURCES), os.cpu_count() or 1))
+    with ThreadPoolExecutor(max_workers=jobs) as ex:
+        objs = list(ex.map(lambda s: _compile(s, verbose), SOURCES))
+    tmp = LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.run([_nvcc(), *ARCH, "-shared", "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB_PATH)
     return LIB_PATH
 

@@ -20,6 +20,7 @@ GEMM_ERR_NO_MEMORY = 5
 
 GEMM_OUT_F32 = 0
 GEMM_OUT_BF16 = 1
+GEMM_OUT_F16 = 2
 
 # Every function declared in include/gemm_bf16.h: (restype, argtypes).
 _I = ctypes.c_int
@@ -36,6 +37,20 @@ SIGNATURES = {
     "gemm_bf16_set_wait_timeout_ns": (_I, [ctypes.c_ulonglong]),
     "gemm_bf16_version": (_I, []),
     "gemm_bf16_noalloc": (_I, [_I, _I, _I, _P, _I, _P, _I, _P, _I, _I, _F, _F, _P]),
+    "gemm_f16": (_I, [_I, _I, _I, _P, _I, _P, _I, _P, _I, _I, _F, _F, _P]),
+    "gemm_f16_batched_shared_w": (_I, [_I, _I, _I, _I, _P, _I, _P, _I, _LL, _P, _I, _LL, _I, _F, _F,
+                                       _P]),
+    "gemm_bf16_batched_shared_w_dedup": (_I, [_I, _I, _I, _I, _I, _P, _I, _P, _I, _LL, _P, _P, _I, _LL, _I,
+                                              _F, _F, _P]),
+    "gemm_autotune": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _I, _LL, _P, _P, _I, _LL, _I, _F, _F, _P,
+                           ctypes.POINTER(ctypes.c_float)]),
+    "gemm_tuning_clear": (_I, []),
+    "gemm_tuning_size": (_I, []),
+    "gemm_tuning_save": (_I, [ctypes.c_char_p]),
+    "gemm_tuning_load": (_I, [ctypes.c_char_p]),
+    "gemm_last_config": (_I, [ctypes.POINTER(_I)] * 4),
+    "gemm_bf16_tensor_map_cache_stats": (_I, [ctypes.POINTER(ctypes.c_ulonglong),
+                                              ctypes.POINTER(ctypes.c_ulonglong)]),
 }
 
 # Size of the fixed device scratch used by gemm_bf16_noalloc (GEMM_BF16_NOALLOC_SCRATCH_BYTES).
@@ -100,3 +115,62 @@ def gemm_bf16_version() -> int:
 def gemm_bf16_noalloc(M, N, K, A, lda, B, ldb, C, ldc, out_type, alpha, beta, stream) -> int:
     """gemm_bf16 without any device allocation (fixed 32 MiB library scratch)."""
     return LIB.gemm_bf16_noalloc(M, N, K, A, lda, B, ldb, C, ldc, out_type, alpha, beta, stream)
+
+
+def gemm_f16(M, N, K, A, lda, B, ldb, C, ldc, out_type, alpha, beta, stream) -> int:
+    return LIB.gemm_f16(M, N, K, A, lda, B, ldb, C, ldc, out_type, alpha, beta, stream)
+
+
+def gemm_f16_batched_shared_w(batch, M, N, K, W, ldw, X, ldx, stride_x, Y, ldy, stride_y, out_type,
+                              alpha, beta, stream) -> int:
+    return LIB.gemm_f16_batched_shared_w(batch, M, N, K, W, ldw, X, ldx, stride_x, Y, ldy, stride_y,
+                                         out_type, alpha, beta, stream)
+
+
+def gemm_bf16_tensor_map_cache_stats() -> tuple[int, int]:
+    """(hits, misses) of the library's tensor-map cache."""
+    h, m = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+    st = LIB.gemm_bf16_tensor_map_cache_stats(ctypes.byref(h), ctypes.byref(m))
+    if st != GEMM_OK:
+        raise GemmError(st, "gemm_bf16_tensor_map_cache_stats")
+    return int(h.value), int(m.value)
+
+
+def gemm_bf16_batched_shared_w_dedup(batch, n_unique, M, N, K, W, ldw, X, ldx, stride_x, index, Y, ldy,
+                                     stride_y, out_type, alpha, beta, stream) -> int:
+    return LIB.gemm_bf16_batched_shared_w_dedup(batch, n_unique, M, N, K, W, ldw, X, ldx, stride_x, index,
+                                                Y, ldy, stride_y, out_type, alpha, beta, stream)
+
+
+def gemm_autotune(in_type, form, batch, n_unique, M, N, K, A, lda, B, ldb, stride_b, index, C, ldc, stride_c,
+                  out_type, alpha, beta, stream) -> tuple[int, float]:
+    """(status, best time per call in us) of the C autotuner."""
+    best = ctypes.c_float(0.0)
+    st = LIB.gemm_autotune(in_type, form, batch, n_unique, M, N, K, A, lda, B, ldb, stride_b, index, C, ldc,
+                           stride_c, out_type, alpha, beta, stream, ctypes.byref(best))
+    return st, float(best.value)
+
+
+def gemm_tuning_clear() -> int:
+    return LIB.gemm_tuning_clear()
+
+
+def gemm_tuning_size() -> int:
+    return LIB.gemm_tuning_size()
+
+
+def gemm_tuning_save(path: str) -> int:
+    return LIB.gemm_tuning_save(path.encode())
+
+
+def gemm_tuning_load(path: str) -> int:
+    return LIB.gemm_tuning_load(path.encode())
+
+
+def gemm_last_config() -> tuple[int, int, int, int]:
+    """(plan, workspace K slices, cluster K slices, raster group) of this thread's last launch."""
+    v = [ctypes.c_int(0) for _ in range(4)]
+    st = LIB.gemm_last_config(*[ctypes.byref(x) for x in v])
+    if st != GEMM_OK:
+        raise GemmError(st, "gemm_last_config")
+    return tuple(int(x.value) for x in v)

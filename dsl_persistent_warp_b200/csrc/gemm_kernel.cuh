@@ -33,12 +33,34 @@
 
 #include "ptx_sm100.cuh"
 
+#ifndef PW_OPERAND_L2_POLICY
+#define PW_OPERAND_L2_POLICY 1
+#endif
+#ifndef PW_SUBTILE_SKEW
+#define PW_SUBTILE_SKEW 1
+#endif
+
 namespace pw {
 
-enum : int { OUT_F32 = 0, OUT_BF16 = 1 };
+enum : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_F16 = 2 };
 
-// Device status word: bit i set = a bounded wait of role i expired (see kStatus*).
-__device__ unsigned int g_pw_status;
+// 16-bit output element <-> fp32.  Packed words hold element 2j in bits 0..15 and element
+// 2j+1 in bits 16..31; both conversions to 16 bits round to nearest even once.
+template <int OUT>
+__device__ __forceinline__ float dec16_lo(uint32_t w) {
+    if constexpr (OUT == OUT_BF16) return __uint_as_float(w << 16);
+    else return f16_to_f32((uint16_t)(w & 0xFFFFu));
+}
+template <int OUT>
+__device__ __forceinline__ float dec16_hi(uint32_t w) {
+    if constexpr (OUT == OUT_BF16) return __uint_as_float(w & 0xFFFF0000u);
+    else return f16_to_f32((uint16_t)(w >> 16));
+}
+template <int OUT>
+__device__ __forceinline__ uint32_t pack16(float lo, float hi) {
+    if constexpr (OUT == OUT_BF16) return pack_bf16x2(lo, hi);
+    else return pack_f16x2(lo, hi);
+}
 
 enum : unsigned int {
     kStatusProducer = 1u,
@@ -67,11 +89,24 @@ struct KParams {
     int batch_real;          // number of batch entries (p.batch counts tile batches)
     int splits;              // K slices per tile (split-K; <= 1: none).  Work unit u covers tile
                              // u / splits and k-blocks [s*kb_per_split, (s+1)*kb_per_split), s = u % splits
-    int kb_per_split;
+    int kb_per_split;        // k-blocks per slice (global or cluster split-K)
+    int csplit;              // cluster split-K (one-CTA plans): K slices per tile, computed by the
+                             // csplit CTAs of one thread-block cluster, one slice each; the partial
+                             // sums are added through distributed shared memory (<= 1: none)
     float* ws;               // split-K partials: per (tile, CTA rank, slice) the CTA's 128 rows x
                              // TILE_N columns in fp32, as 4 KiB pieces per epilogue warp
     unsigned int* counters;  // split-K arrivals per (tile, CTA rank, epilogue warp); zero on entry,
                              // and the last arrival puts it back to zero
+    // Deduplicated batches (shared-W form): the tiles cover the batch_real distinct X entries;
+    // the result of entry e goes to the items dd_dst[dd_off[e] .. dd_off[e+1]) of the output
+    // (Y has `batch_out` entries).  Each tile is computed by `dsplit` work units, unit part k
+    // storing destinations k, k + dsplit, ... of each entry (nullptr: no deduplication).
+    const int* dd_off;
+    const int* dd_dst;
+    int dsplit;
+    int batch_out;
+    unsigned int* status;    // device status word: bit i set = a bounded wait of role i expired
+    int in_f16;              // 1: A and B hold fp16 values, 0: bf16
     int test_stall;          // test hook: the producer issues nothing, so the first bounded
                              // wait of the MMA thread expires (failure-detection tests)
     unsigned long long timeout_ns;
@@ -132,6 +167,10 @@ struct Tile {
     static constexpr int MN_BOX_BYTES = 64 * 2 * BK;
     static_assert(BK == 64 || BK == 32, "stage K");
     static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
+    // Cluster split-K: after its K slice, a CTA's ring is idle and holds its 128 x BN fp32
+    // partial tile for the other CTAs of the cluster to read.
+    static constexpr int XCHG_BYTES = 128 * BN * 4;
+    static constexpr bool CSPLIT_OK = CG == 1 && NSUB == 1 && ARES == 0 && XCHG_BYTES <= STAGES * STAGE_BYTES;
     static_assert(ARES == 0 || BK == 64, "resident A uses K=64 blocks");
 };
 
@@ -151,8 +190,9 @@ __device__ __forceinline__ void decode_tile(const KParams& p, int t, int& b, int
 }
 
 template <int CG>
-__device__ __forceinline__ void raise_abort(uint32_t slot_abort, uint32_t rank, unsigned int code) {
-    atomicOr(&g_pw_status, code);
+__device__ __forceinline__ void raise_abort(uint32_t slot_abort, uint32_t rank, unsigned int* status,
+                                            unsigned int code) {
+    atomicOr(status, code);
     st_shared_volatile_u32(slot_abort, 1u);
     if constexpr (CG == 2) st_cluster_u32(map_to_rank(slot_abort, rank ^ 1u), 1u);
 }
@@ -160,8 +200,8 @@ __device__ __forceinline__ void raise_abort(uint32_t slot_abort, uint32_t rank, 
 // Slow path of wait_phase: poll with the global-timer bound.
 template <int CG, bool CLUSTER_SCOPE>
 __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, uint32_t slot_abort,
-                                             uint32_t rank, unsigned long long timeout_ns,
-                                             unsigned int code) {
+                                             uint32_t rank, unsigned int* status,
+                                             unsigned long long timeout_ns, unsigned int code) {
     const uint64_t t0 = global_timer_ns();
     for (;;) {
 #pragma unroll 1
@@ -170,7 +210,7 @@ __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, uint
                 return true;
         if (ld_shared_volatile_u32(slot_abort) != 0u) return false;
         if (global_timer_ns() - t0 > timeout_ns) {
-            raise_abort<CG>(slot_abort, rank, code);
+            raise_abort<CG>(slot_abort, rank, status, code);
             return false;
         }
     }
@@ -181,10 +221,10 @@ __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, uint
 // critical path (a stage that is already full or free) it costs one instruction.
 template <int CG, bool CLUSTER_SCOPE>
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint32_t slot_abort,
-                                           uint32_t rank, unsigned long long timeout_ns,
-                                           unsigned int code) {
+                                           uint32_t rank, unsigned int* status,
+                                           unsigned long long timeout_ns, unsigned int code) {
     if (CLUSTER_SCOPE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    return wait_phase_slow<CG, CLUSTER_SCOPE>(bar, parity, slot_abort, rank, timeout_ns, code);
+    return wait_phase_slow<CG, CLUSTER_SCOPE>(bar, parity, slot_abort, rank, status, timeout_ns, code);
 }
 
 template <int CG, int BN, int NSUB, int STAGES, int BK, int B_MN, int OUT, int ARES>
@@ -200,8 +240,23 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
     const uint32_t warp = threadIdx.x >> 5;
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
-    const int cluster_id = blockIdx.x / CG;
-    const int num_clusters = gridDim.x / CG;
+    // Cluster split-K: the grid holds one cluster of CS CTAs per tile; CTA crank of the cluster
+    // computes K slice crank of the tile.  Otherwise a persistent grid of CG-CTA clusters.
+    const int CS = (T::CSPLIT_OK && p.csplit > 1) ? p.csplit : 1;
+    const uint32_t crank = CS > 1 ? cluster_ctarank() : 0u;
+    const int cluster_id = CS > 1 ? (int)(blockIdx.x / CS) : (int)(blockIdx.x / CG);
+    const int num_clusters = CS > 1 ? (int)(gridDim.x / CS) : (int)(gridDim.x / CG);
+    // K blocks of work unit u (global split-K: unit = (tile, slice); cluster split-K: this CTA's
+    // slice of the tile; else all of K).
+    const int SG = (ARES == 0 && p.splits > 1) ? p.splits : 1;
+    // Work units per tile: global split-K slices, or the deduplicated form's destination parts.
+    const int DS = (p.dd_off != nullptr && p.dsplit > 1) ? p.dsplit : 1;
+    const int UPT = SG > 1 ? SG : DS;
+    auto unit_k = [&](int u, int& kb_lo, int& kb_hi) {
+        const int sl = SG > 1 ? u % SG : (int)crank;
+        kb_lo = (SG > 1 || CS > 1) ? sl * p.kb_per_split : 0;
+        kb_hi = (SG > 1 || CS > 1) ? min(p.k_blocks, kb_lo + p.kb_per_split) : p.k_blocks;
+    };
 
     const uint32_t bar0 = sbase + T::OFF_BAR;
     auto bar_full = [&](int s) { return bar0 + 8u * s; };
@@ -243,8 +298,15 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint32_t full_leader0 = CG == 2 ? map_to_rank(bar_full(0), 0) : bar_full(0);
-            // A and B panels are read by several CTAs of a wave: keep them in L2.
+            // A and B panels are read by several CTAs of a wave: keep them in L2 (build option
+            // PW_OPERAND_L2_POLICY: 0 evict-normal, 1 evict-last, 2 evict-first).
+#if PW_OPERAND_L2_POLICY == 0
+            const uint64_t pol = l2_policy_evict_normal();
+#elif PW_OPERAND_L2_POLICY == 2
+            const uint64_t pol = l2_policy_evict_first();
+#else
             const uint64_t pol = l2_policy_evict_last();
+#endif
             int stage = 0;
             uint32_t phase = 0;
             bool ok = p.test_stall == 0;
@@ -258,17 +320,17 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     else tma_load_3d_pair(sa, &tmA, ares_bar, kb * T::BK, (int)rank * 128, 0, pol);
                 }
             }
-            const int S = (ARES == 0 && p.splits > 1) ? p.splits : 1;  // split-K: streaming plans only
+            const int S = UPT;
             for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters) {
                 const int t = u / S;
-                const int kb_lo = S > 1 ? (u % S) * p.kb_per_split : 0;
-                const int kb_hi = S > 1 ? min(p.k_blocks, kb_lo + p.kb_per_split) : p.k_blocks;
+                int kb_lo, kb_hi;
+                unit_k(u, kb_lo, kb_hi);
                 int b, mb, nb;
                 decode_tile(p, t, b, mb, nb);
                 const int a_row = mb * T::BM + (int)rank * 128;
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!wait_phase<CG, false>(bar_empty(stage), phase ^ 1u, slot_abort, rank,
-                                               p.timeout_ns, kStatusProducer)) {
+                                               p.status, p.timeout_ns, kStatusProducer)) {
                         ok = false;
                         break;
                     }
@@ -310,7 +372,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t IDESC = idesc_bf16_f32(T::BM, BN, 0, B_MN);
+            const uint32_t IDESC = idesc_f16_kind(T::BM, BN, 0, B_MN, p.in_f16);
             // Descriptors of stage 0 (K step 0); other stages and K steps only add to the
             // start-address field, which never carries out of its 14 bits (smem < 256 KiB).
             const uint64_t adesc0 = smem_desc(sbase + T::OFF_A, 16, T::KMAJ_SBO, T::KMAJ_SWIZZLE);
@@ -326,15 +388,120 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             int acc = 0;                 // slot of the tile when NSUB == 1
             bool ok = true;
             if constexpr (ARES != 0) {
-                ok = wait_phase<CG, false>(bar_ares, 0u, slot_abort, rank, p.timeout_ns, kStatusMma);
+                ok = wait_phase<CG, false>(bar_ares, 0u, slot_abort, rank, p.status, p.timeout_ns, kStatusMma);
                 tc_fence_after();
             }
-            const int S = (ARES == 0 && p.splits > 1) ? p.splits : 1;  // split-K: streaming plans only
+            const int S = UPT;
+            auto commit_tfull = [&](int slot) {
+                // accumulator of this slot complete: hand it to the epilogue
+                if constexpr (CG == 1) {
+                    umma_commit<1>(bar_tfull(slot));
+                } else {
+                    umma_commit<2>(tfull_r0 + 8u * slot);
+                    umma_commit<2>(tfull_r1 + 8u * slot);
+                }
+            };
+            auto commit_empty = [&](int st) {
+                if constexpr (CG == 1) {
+                    umma_commit<1>(bar_empty(st));
+                } else {
+                    umma_commit<2>(empty_r0 + 8u * st);
+                    umma_commit<2>(empty_r1 + 8u * st);
+                }
+            };
+            if constexpr (NSUB == 2 && ARES == 0 && PW_SUBTILE_SKEW) {
+                // Two sub-tiles own both accumulator slots, so a tile's epilogue would hold up the
+                // next tile's first k-block.  Sub-tile 1 may instead trail sub-tile 0 by up to
+                // STAGES k-blocks, whose stages stay held until its MMAs are issued:
+                //  * in a unit's last STAGES-1 k-blocks sub-tile 1 waits, so sub-tile 0 -- and the
+                //    drain of slot 0 -- finish while sub-tile 1 completes the unit;
+                //  * at a unit's start, while slot 1 is still being drained, sub-tile 0 runs ahead.
+                // The queue of held stages lives in one register: per entry 8 bits -- stage (0-2),
+                // first k-block of its unit (3), last (4), in the unit's tail (5), unit tag (6-7).
+                static_assert(STAGES <= 8, "stage index in 3 bits");
+                uint64_t pq = 0;
+                int qn = 0;
+                auto mma_sub = [&](int sub, int st, bool first) {
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(sub * BN);
+                    const uint64_t a_st = adesc0 + (uint64_t)((st * T::A_BYTES) >> 4);
+                    const uint64_t b_sub = bdesc0 + (uint64_t)((st * T::B_BYTES + sub * T::B_SUB_BYTES) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < T::BK / 16; ++kk)
+                        umma_f16<CG>(d_tmem, a_st + (uint64_t)((kk * 32) >> 4),
+                                     b_sub + (uint64_t)((B_MN ? kk * 2048 : kk * 32) >> 4), IDESC,
+                                     (!first || kk != 0) ? 1u : 0u);
+                };
+                // sub-tile 1 of the oldest held stage; false when a wait gave up
+                auto pop_sub1 = [&]() -> bool {
+                    const uint32_t e = (uint32_t)(pq & 0xFFu);
+                    if (e & 8u) {
+                        if (!wait_phase<CG, CG == 2>(bar_tempty(1), ((tph >> 1) & 1u) ^ 1u, slot_abort, rank,
+                                                     p.status, p.timeout_ns, kStatusMma))
+                            return false;
+                        tc_fence_after();
+                        tph ^= 2u;
+                    }
+                    mma_sub(1, (int)(e & 7u), (e & 8u) != 0u);
+                    if (e & 16u) commit_tfull(1);
+                    commit_empty((int)(e & 7u));
+                    pq >>= 8;
+                    --qn;
+                    return true;
+                };
+                uint32_t utag = 0;  // unit counter mod 4
+                for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters, utag = (utag + 1) & 3u) {
+                    int kb_lo, kb_hi;
+                    unit_k(u, kb_lo, kb_hi);
+                    // Slot 0's drain for this unit needs the epilogue past the unit before the
+                    // previous one: issue what is still held from those older units.
+                    while (ok && qn > 0 && (((utag - (uint32_t)(pq >> 6)) & 3u) >= 2u)) ok = pop_sub1();
+                    for (int kb = kb_lo; ok && kb < kb_hi; ++kb) {
+                        if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, rank, p.status, p.timeout_ns,
+                                                   kStatusMma)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        if (kb == kb_lo) {
+                            if (!wait_phase<CG, CG == 2>(bar_tempty(0), (tph & 1u) ^ 1u, slot_abort, rank, p.status,
+                                                         p.timeout_ns, kStatusMma)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            tph ^= 1u;
+                        }
+                        mma_sub(0, stage, kb == kb_lo);
+                        if (kb == kb_hi - 1) commit_tfull(0);
+                        const uint32_t e = (uint32_t)stage | (kb == kb_lo ? 8u : 0u) | (kb == kb_hi - 1 ? 16u : 0u) |
+                                           (kb >= kb_hi - (STAGES - 1) ? 32u : 0u) | (utag << 6);
+                        pq |= (uint64_t)e << (8 * qn);
+                        ++qn;
+                        while (ok && qn > 0) {
+                            if (qn < STAGES) {
+                                const uint32_t f = (uint32_t)(pq & 0xFFu);
+                                // slot 1 still being drained: let sub-tile 0 run ahead
+                                if ((f & 8u) && !(CG == 2 ? mbar_test_wait_cluster(bar_tempty(1), ((tph >> 1) & 1u) ^ 1u)
+                                                          : mbar_test_wait(bar_tempty(1), ((tph >> 1) & 1u) ^ 1u)))
+                                    break;
+                                // the unit's tail: hold sub-tile 1 back until sub-tile 0 has finished
+                                if ((f & 32u) && (f >> 6) == utag && kb < kb_hi - 1) break;
+                            }
+                            ok = pop_sub1();
+                        }
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+                while (ok && qn > 0) ok = pop_sub1();
+            } else {
             for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters) {
-                const int kb_lo = S > 1 ? (u % S) * p.kb_per_split : 0;
-                const int kb_hi = S > 1 ? min(p.k_blocks, kb_lo + p.kb_per_split) : p.k_blocks;
+                int kb_lo, kb_hi;
+                unit_k(u, kb_lo, kb_hi);
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
-                    if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, rank, p.timeout_ns,
+                    if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, rank, p.status, p.timeout_ns,
                                                kStatusMma)) {
                         ok = false;
                         break;
@@ -349,7 +516,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                         if (kb == kb_lo) {
                             // the slot must have been drained by the epilogue of its last use
                             if (!wait_phase<CG, CG == 2>(bar_tempty(slot), ((tph >> slot) & 1u) ^ 1u, slot_abort, rank,
-                                                         p.timeout_ns, kStatusMma)) {
+                                                         p.status, p.timeout_ns, kStatusMma)) {
                                 ok = false;
                                 break;
                             }
@@ -364,23 +531,10 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                             const uint64_t bdesc = b_sub + (uint64_t)((B_MN ? kk * 2048 : kk * 32) >> 4);
                             umma_f16<CG>(d_tmem, adesc, bdesc, IDESC, (kb != kb_lo || kk != 0) ? 1u : 0u);
                         }
-                        if (kb == kb_hi - 1) {
-                            // accumulator of this slot complete: hand it to the epilogue
-                            if constexpr (CG == 1) {
-                                umma_commit<1>(bar_tfull(slot));
-                            } else {
-                                umma_commit<2>(tfull_r0 + 8u * slot);
-                                umma_commit<2>(tfull_r1 + 8u * slot);
-                            }
-                        }
+                        if (kb == kb_hi - 1) commit_tfull(slot);
                     }
                     if (!ok) break;
-                    if constexpr (CG == 1) {
-                        umma_commit<1>(bar_empty(stage));
-                    } else {
-                        umma_commit<2>(empty_r0 + 8u * stage);
-                        umma_commit<2>(empty_r1 + 8u * stage);
-                    }
+                    commit_empty(stage);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -392,6 +546,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 } else {
                     tph ^= 3u;
                 }
+            }
             }
         }
     } else {
@@ -408,20 +563,25 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         bool ok = true;
         // alpha/beta, conversion and store of chunk c (STG_COLS columns) of sub-tile `sub` of the
         // tile (b, nb) for the 32-row slab starting at row0; v holds this lane's row.
-        auto finish_chunk = [&](int b, int nb, int row0, int row, int sub, int c, float (&v)[T::STG_COLS]) {
+        // bout >= 0: store to output entry bout instead of the chunk's own batch entry (the
+        // deduplicated form's scatter; C_in is read from the same entry).
+        auto finish_chunk = [&](int b, int nb, int row0, int row, int sub, int c, float (&v)[T::STG_COLS],
+                                int bout = -1) {
             const int col_tile = sub * T::BN_CTA;  // column within the tile
             const int jc = c * T::STG_COLS;
             const int tcol = col_tile + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
-            const int bb = p.pack > 1 ? nb * p.pack + tcol / p.N : b;
+            const int bsrc = p.pack > 1 ? nb * p.pack + tcol / p.N : b;
+            // a chunk beyond the last entry stores nothing; otherwise bb is the output entry
+            const bool entry_in = bsrc < p.batch_real;
+            const int bb = !entry_in ? p.batch_real : bout >= 0 ? bout : bsrc;
             const int colc = p.pack > 1 ? tcol % p.N : nb * T::TILE_N + tcol;
             const long long cbase = (long long)bb * p.stride_c + (long long)row * p.ldc;
-            const bool row_in = row < p.M && bb < p.batch_real;
+            const bool row_in = row < p.M && entry_in;
             const bool full_cols = colc + T::STG_COLS <= p.N;
             // A chunk goes out as one tensor store when C is TMA-addressable up to the
             // chunk's end; otherwise (unaligned ldc, a ragged right edge) the warp moves it
             // row by row through the staging buffer so that every access is coalesced.
-            const bool tma_chunk =
-                p.c_tma && colc + T::STG_COLS <= p.n_store_tma && bb < p.batch_real;
+            const bool tma_chunk = p.c_tma && colc + T::STG_COLS <= p.n_store_tma && entry_in;
             const bool coop_chunk = !tma_chunk;
             const uint32_t sbuf = stg + buf * T::STG_BYTES;
             // the buffer may still be read by an earlier tensor store
@@ -435,9 +595,9 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 // go RB at a time so that RB (2 RB for bf16) loads per lane are in flight:
                 // 16 rows keep the register budget of the other paths (32 spill).
                 constexpr int RB = 16;
-                constexpr int EPR = OUT == OUT_BF16 ? 2 : 1;  // elements per lane and row
-                constexpr int ES = OUT == OUT_BF16 ? 2 : 4;   // bytes per element
-                const int nrows = bb < p.batch_real ? min(32, p.M - row0) : 0;
+                constexpr int EPR = OUT != OUT_F32 ? 2 : 1;  // elements per lane and row
+                constexpr int ES = OUT != OUT_F32 ? 2 : 4;   // bytes per element
+                const int nrows = entry_in ? min(32, p.M - row0) : 0;
                 const char* src = static_cast<const char*>(p.C) +
                                   ((long long)bb * p.stride_c + (long long)row0 * p.ldc + colc + (int)lane) * ES;
                 const long long sstep = (long long)p.ldc * ES;
@@ -455,7 +615,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                         for (int h = 0; h < EPR; ++h) {
                             x[i * EPR + h] = 0u;
                             if (rv && ev[h]) {
-                                if constexpr (OUT == OUT_BF16)
+                                if constexpr (OUT != OUT_F32)
                                     x[i * EPR + h] = *reinterpret_cast<const uint16_t*>(rp + 64 * h);
                                 else
                                     x[i * EPR + h] = *reinterpret_cast<const uint32_t*>(rp);
@@ -469,7 +629,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
 #pragma unroll
                         for (int h = 0; h < EPR; ++h) {
                             const int e = (int)lane + 32 * h;
-                            if constexpr (OUT == OUT_BF16)
+                            if constexpr (OUT != OUT_F32)
                                 st_shared_u16(srow + ((uint32_t)((e >> 3) ^ (r & 7)) << 4) + (uint32_t)(e & 7) * 2u,
                                               (uint16_t)x[i * EPR + h]);
                             else
@@ -488,11 +648,10 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                         const uint32_t xs[4] = {x0, x1, x2, x3};
 #pragma unroll
                         for (int h = 0; h < 4; ++h) {
-                            if constexpr (OUT == OUT_BF16) {
+                            if constexpr (OUT != OUT_F32) {
                                 const int e = 8 * cc + 2 * h;
-                                if (colc + e < p.N) v[e] = fmaf(p.beta, __uint_as_float(xs[h] << 16), v[e]);
-                                if (colc + e + 1 < p.N)
-                                    v[e + 1] = fmaf(p.beta, __uint_as_float(xs[h] & 0xFFFF0000u), v[e + 1]);
+                                if (colc + e < p.N) v[e] = fmaf(p.beta, dec16_lo<OUT>(xs[h]), v[e]);
+                                if (colc + e + 1 < p.N) v[e + 1] = fmaf(p.beta, dec16_hi<OUT>(xs[h]), v[e + 1]);
                             } else {
                                 const int e = 4 * cc + h;
                                 if (colc + e < p.N) v[e] = fmaf(p.beta, __uint_as_float(xs[h]), v[e]);
@@ -503,7 +662,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 __syncwarp();  // every lane has its C_in before the buffer is overwritten
             } else if (p.c_read && row_in) {
                 if (full_cols && p.c_tma) {
-                    if constexpr (OUT == OUT_BF16) {
+                    if constexpr (OUT != OUT_F32) {
                         const uint4* src = reinterpret_cast<const uint4*>(
                             static_cast<const uint16_t*>(p.C) + cbase + colc);
 #pragma unroll
@@ -512,10 +671,8 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                             for (int h = 0; h < 4; ++h) {
-                                v[8 * j + 2 * h] =
-                                    fmaf(p.beta, __uint_as_float(ww[h] << 16), v[8 * j + 2 * h]);
-                                v[8 * j + 2 * h + 1] = fmaf(
-                                    p.beta, __uint_as_float(ww[h] & 0xFFFF0000u), v[8 * j + 2 * h + 1]);
+                                v[8 * j + 2 * h] = fmaf(p.beta, dec16_lo<OUT>(ww[h]), v[8 * j + 2 * h]);
+                                v[8 * j + 2 * h + 1] = fmaf(p.beta, dec16_hi<OUT>(ww[h]), v[8 * j + 2 * h + 1]);
                             }
                         }
                     } else {
@@ -535,9 +692,8 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     for (int j = 0; j < T::STG_COLS; ++j) {
                         if (colc + j < p.N) {
                             float cin;
-                            if constexpr (OUT == OUT_BF16)
-                                cin = __uint_as_float(
-                                    (uint32_t)(static_cast<const uint16_t*>(p.C)[cbase + colc + j]) << 16);
+                            if constexpr (OUT != OUT_F32)
+                                cin = dec16_lo<OUT>(static_cast<const uint16_t*>(p.C)[cbase + colc + j]);
                             else
                                 cin = static_cast<const float*>(p.C)[cbase + colc + j];
                             v[j] = fmaf(p.beta, cin, v[j]);
@@ -547,9 +703,9 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             }
             // pack the 128-byte row segment into 8 x 16-byte words
             uint32_t w[32];
-            if constexpr (OUT == OUT_BF16) {
+            if constexpr (OUT != OUT_F32) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                for (int j = 0; j < 32; ++j) w[j] = pack16<OUT>(v[2 * j], v[2 * j + 1]);
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
@@ -574,15 +730,15 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     // one shared load and one store per element (the loop is issue-bound: one
                     // warp per scheduler, nothing else to hide latency behind).
                     __syncwarp();
-                    constexpr int ES = OUT == OUT_BF16 ? 2 : 4;  // bytes per element
-                    constexpr int EPR = OUT == OUT_BF16 ? 2 : 1;  // elements per lane and row
-                    const int nrows = bb < p.batch_real ? min(32, p.M - row0) : 0;
+                    constexpr int ES = OUT != OUT_F32 ? 2 : 4;  // bytes per element
+                    constexpr int EPR = OUT != OUT_F32 ? 2 : 1;  // elements per lane and row
+                    const int nrows = entry_in ? min(32, p.M - row0) : 0;
                     char* dst = static_cast<char*>(p.C) +
                                 ((long long)bb * p.stride_c + (long long)row0 * p.ldc + colc + (int)lane) * ES;
                     const long long dstep = (long long)p.ldc * ES;
                     bool ev[EPR];
                     uint32_t ch[EPR];
-                    const uint32_t inb = OUT == OUT_BF16 ? (lane & 7u) * 2u : (lane & 3u) * 4u;
+                    const uint32_t inb = OUT != OUT_F32 ? (lane & 7u) * 2u : (lane & 3u) * 4u;
 #pragma unroll
                     for (int h = 0; h < EPR; ++h) {
                         const int e = (int)lane + 32 * h;
@@ -597,7 +753,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                         for (int h = 0; h < EPR; ++h) {
                             if (!ev[h]) continue;
                             const uint32_t a = srow + ((ch[h] ^ sw) << 4);
-                            if constexpr (OUT == OUT_BF16)
+                            if constexpr (OUT != OUT_F32)
                                 *reinterpret_cast<uint16_t*>(dst + 64 * h) = ld_shared_u16(a);
                             else
                                 *reinterpret_cast<uint32_t*>(dst) = ld_shared_u32(a);
@@ -612,7 +768,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         auto load_chunk = [&](uint32_t trow, int c, float (&v)[T::STG_COLS]) {
             uint32_t r0[32];
             tmem_ld_32x32b_x32(trow + c * T::STG_COLS, r0);
-            if constexpr (OUT == OUT_BF16) {
+            if constexpr (OUT != OUT_F32) {
                 uint32_t r1[32];
                 tmem_ld_32x32b_x32(trow + c * T::STG_COLS + 32, r1);
                 tmem_ld_wait(r0);
@@ -647,10 +803,20 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             }
             __syncwarp();
         };
-        const int S = (ARES == 0 && p.splits > 1) ? p.splits : 1;  // split-K: streaming plans only
-        for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters) {
-            const int t = u / S;
-            const int sl = u % S;
+        const int S = SG;  // global split-K: streaming plans only
+        // Cluster split-K exchange buffer: the ring, as 4 KiB pieces (32 rows x 32 fp32 columns,
+        // the staging-buffer image), piece (32-column block cb, lane quarter qq) at
+        // ((cb * 4 + qq) << 12).
+        const uint32_t xchg = sbase + T::OFF_A;
+        // batch entry of chunk c of sub-tile `sub` of tile (b, nb) (several per tile when packed)
+        auto chunk_entry = [&](int b, int nb, int sub, int c) {
+            const int jc = c * T::STG_COLS;
+            const int tcol = sub * T::BN_CTA + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
+            return p.pack > 1 ? nb * p.pack + tcol / p.N : b;
+        };
+        for (int u = cluster_id; ok && u < p.tiles * UPT; u += num_clusters) {
+            const int t = u / UPT;
+            const int sl = u % UPT;  // split-K slice, or destination part of a deduplicated batch
             int b, mb, nb;
             decode_tile(p, t, b, mb, nb);
             const int row0 = mb * T::BM + (int)rank * 128 + 32 * q;
@@ -666,7 +832,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 const int slot = NSUB == 1 ? acc : sub;
                 int w_ok = 1;
                 if (lane == 0)
-                    w_ok = wait_phase<CG, false>(bar_tfull(slot), (tph >> slot) & 1u, slot_abort, rank, p.timeout_ns,
+                    w_ok = wait_phase<CG, false>(bar_tfull(slot), (tph >> slot) & 1u, slot_abort, rank, p.status, p.timeout_ns,
                                                  kStatusEpilogue);
                 w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
                 if (!w_ok) {
@@ -681,7 +847,19 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     const int c = half * CPW + ci;
                     float v[T::STG_COLS];
                     load_chunk(trow, c, v);
-                    if (S == 1) {
+                    if (CS > 1) {
+                        // this CTA's K-slice partial sums, for the cluster's reduction below
+                        if (ci == 0) fence_proxy_async_smem();
+#pragma unroll
+                        for (int h = 0; h < PIECES; ++h) {
+                            const uint32_t pc = xchg + ((uint32_t)((c * PIECES + h) * 4 + q) << 12) + lane * 128u;
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                st_shared_v4(pc + ((uint32_t)(j ^ (int)(lane & 7u)) << 4), __float_as_uint(v[32 * h + 4 * j]),
+                                             __float_as_uint(v[32 * h + 4 * j + 1]), __float_as_uint(v[32 * h + 4 * j + 2]),
+                                             __float_as_uint(v[32 * h + 4 * j + 3]));
+                        }
+                    } else if (S == 1 && p.dd_off == nullptr) {
                         if (ci == CPW - 1) {
                             // Slot drained: hand it back to the MMA warp (leader CTA).
                             tc_fence_before();
@@ -689,6 +867,29 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                             if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * slot);
                         }
                         finish_chunk(b, nb, row0, row, sub, c, v);
+                    } else if (S == 1) {
+                        // Deduplicated batch: the chunk's distinct entry goes to every item that
+                        // uses it; this unit stores destinations sl, sl + DS, ... of the entry's
+                        // list, reloading the accumulator from TMEM for each one.  The slot is
+                        // handed back after the last reload of the warp's last chunk.
+                        const int e = chunk_entry(b, nb, sub, c);
+                        int k = 0, hi = 0;
+                        if (e < p.batch_real) {
+                            k = __ldg(p.dd_off + e) + sl;
+                            hi = __ldg(p.dd_off + e + 1);
+                        }
+                        auto release = [&]() {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * slot);
+                        };
+                        if (k >= hi && ci == CPW - 1) release();
+                        for (bool first = true; k < hi; k += DS, first = false) {
+                            const int d = __ldg(p.dd_dst + k);
+                            if (!first) load_chunk(trow, c, v);
+                            if (ci == CPW - 1 && k + DS >= hi) release();
+                            finish_chunk(b, nb, row0, row, sub, c, v, d);
+                        }
                     } else {
                         // publish this slice's partial sums; the slot stays held for the fixup
                         float* g = slab(sl) + (size_t)((sub * CPW + ci) * PIECES) * 1024;
@@ -780,7 +981,54 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             }
             if (NSUB == 1) acc ^= 1;
         }
+        if constexpr (T::CSPLIT_OK) {
+            if (CS > 1) {
+                // Cluster split-K reduction.  Once every CTA of the cluster has its partial tile in
+                // its shared memory, the cluster's 4*CS epilogue warps share the tile's (lane quarter,
+                // column chunk) items; each adds the CS partials of its item in slice order
+                // 0..CS-1, reading them through distributed shared memory, and runs the normal
+                // alpha/beta epilogue on the sum.  The result does not depend on timing.
+                __syncwarp();
+                cluster_sync();
+                if (ok && ld_shared_volatile_u32(slot_abort) == 0u) {
+                    int b, mb, nb;
+                    decode_tile(p, cluster_id, b, mb, nb);
+                    constexpr int CH = BN / T::STG_COLS;  // column chunks of the tile
+                    for (int it = (int)crank * 4 + ew; it < 4 * CH; it += 4 * CS) {
+                        const int qq = it & 3, c = it >> 2;
+                        const int row0 = mb * T::BM + 32 * qq;
+                        float v[T::STG_COLS];
+#pragma unroll 1
+                        for (int s2 = 0; s2 < CS; ++s2) {
+                            const uint32_t src = map_to_rank(xchg, (uint32_t)s2) + lane * 128u;
+#pragma unroll
+                            for (int h = 0; h < PIECES; ++h) {
+                                uint32_t x[8][4];
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    ld_cluster_v4(src + ((uint32_t)((c * PIECES + h) * 4 + qq) << 12) +
+                                                      ((uint32_t)(j ^ (int)(lane & 7u)) << 4),
+                                                  x[j][0], x[j][1], x[j][2], x[j][3]);
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const float f = __uint_as_float(x[j][e]);
+                                        v[32 * h + 4 * j + e] = s2 == 0 ? f : v[32 * h + 4 * j + e] + f;
+                                    }
+                            }
+                        }
+                        finish_chunk(b, nb, row0, row0 + (int)lane, 0, c, v);
+                    }
+                }
+            }
+        }
         if (p.c_tma && lane == 0) bulk_wait_group_all();
+    }
+    // Producer and MMA warps meet the epilogue's cluster barrier (all partial tiles written).
+    if (CS > 1 && warp < 2) {
+        __syncwarp();
+        cluster_sync();
     }
 
     // ---------------------------------------------------------------- teardown
@@ -791,84 +1039,11 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 5000000ull) nanosleep_ns(100000);
     }
-    if constexpr (CG == 2) cluster_sync(); else __syncthreads();
+    // (cluster split-K: no CTA leaves while another may still read its shared memory)
+    if (CG == 2 || CS > 1) cluster_sync(); else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc<CG>(tmem_base, T::TMEM_COLS);
-    }
-}
-
-// C = beta * C (C = 0 when beta == 0) over batch x M x N: the K == 0 / alpha == 0 case.
-template <typename TC>
-__global__ void scale_c_kernel(TC* C, long long ldc, long long stride_c, int batch, int M, int N,
-                               float beta) {
-    const long long per = (long long)M * N;
-    const long long total = per * batch;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        const long long b = i / per;
-        const long long r = (i - b * per) / N;
-        const long long c = i - b * per - r * N;
-        TC* e = C + b * stride_c + r * ldc + c;
-        float x = 0.0f;
-        if constexpr (sizeof(TC) == 2) {
-            if (beta != 0.0f) x = beta * __uint_as_float((uint32_t)(*reinterpret_cast<uint16_t*>(e)) << 16);
-            *reinterpret_cast<uint16_t*>(e) = (uint16_t)(pack_bf16x2(x, 0.0f) & 0xFFFFu);
-        } else {
-            if (beta != 0.0f) x = beta * *reinterpret_cast<float*>(e);
-            *reinterpret_cast<float*>(e) = x;
-        }
-    }
-}
-
-// Copy a batch x rows x cols bf16 array into a buffer whose leading dimension is a multiple
-// of 8 elements and whose base is 16-byte aligned, so that TMA can read it.  Each thread writes
-// 8 elements with one 16-byte store.  Interior threads read the two aligned 16-byte words that
-// cover their (2-byte aligned) source window and realign them with byte permutes; threads whose
-// aligned window would reach outside [src_lo, src_hi) -- the source allocation's extent -- and
-// row tails use 2-byte loads.
-__global__ void pad_copy_kernel(const uint16_t* __restrict__ src, long long ld_src, long long bs_src,
-                                uint16_t* __restrict__ dst, long long ld_dst, long long bs_dst,
-                                int batch, int rows, int cols, uintptr_t src_lo, uintptr_t src_hi) {
-    const int vec_per_row = (cols + 7) >> 3;
-    for (int b = blockIdx.z; b < batch; b += gridDim.z) {
-        for (int r = blockIdx.y; r < rows; r += gridDim.y) {
-            const uint16_t* s = src + b * bs_src + (long long)r * ld_src;
-            uint16_t* d = dst + b * bs_dst + (long long)r * ld_dst;
-            for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vec_per_row;
-                 v += gridDim.x * blockDim.x) {
-                const int c = v << 3;
-                if (c + 8 <= cols) {
-                    const uintptr_t a = reinterpret_cast<uintptr_t>(s + c);
-                    const uintptr_t a0 = a & ~(uintptr_t)15;
-                    const uint32_t sh = (uint32_t)(a - a0);  // 0, 2, ..., 14
-                    uint32_t e[4];
-                    if (a0 >= src_lo && a0 + 32 <= src_hi) {
-                        const uint4 lo = *reinterpret_cast<const uint4*>(a0);
-                        const uint4 hi = sh ? *reinterpret_cast<const uint4*>(a0 + 16) : lo;
-                        // y[j] = word (sh/4 + j) of the 32-byte window, selected without indexing
-                        const uint32_t wo = sh >> 2;
-                        const uint32_t y0 = wo == 0 ? lo.x : wo == 1 ? lo.y : wo == 2 ? lo.z : lo.w;
-                        const uint32_t y1 = wo == 0 ? lo.y : wo == 1 ? lo.z : wo == 2 ? lo.w : hi.x;
-                        const uint32_t y2 = wo == 0 ? lo.z : wo == 1 ? lo.w : wo == 2 ? hi.x : hi.y;
-                        const uint32_t y3 = wo == 0 ? lo.w : wo == 1 ? hi.x : wo == 2 ? hi.y : hi.z;
-                        const uint32_t y4 = wo == 0 ? hi.x : wo == 1 ? hi.y : wo == 2 ? hi.z : hi.w;
-                        const uint32_t sel = (sh & 2) ? 0x5432u : 0x3210u;  // half-word shift or none
-                        e[0] = __byte_perm(y0, y1, sel);
-                        e[1] = __byte_perm(y1, y2, sel);
-                        e[2] = __byte_perm(y2, y3, sel);
-                        e[3] = __byte_perm(y3, y4, sel);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            e[j] = (uint32_t)s[c + 2 * j] | ((uint32_t)s[c + 2 * j + 1] << 16);
-                    }
-                    *reinterpret_cast<uint4*>(d + c) = make_uint4(e[0], e[1], e[2], e[3]);
-                } else {
-                    for (int j = c; j < cols; ++j) d[j] = s[j];
-                }
-            }
-        }
     }
 }
 

@@ -93,6 +93,32 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     return ok != 0;
 }
 
+// Non-blocking probe of a phase (no suspension); cluster-scope acquire for barriers that
+// receive arrivals from the peer CTA.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // ---------------------------------------------------------------- TMA (bulk tensor)
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
@@ -276,22 +302,36 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
     return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A and B, fp32 D.
+// Instruction descriptor for kind::f16 (16-bit A and B of one type, fp32 D).
 // a_mn / b_mn: 1 when that operand is MN-major in shared memory (0 = K-major).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
-    return (1u << 4)                               // D format: f32
-           | (1u << 7)                             // A format: bf16
-           | (1u << 10)                            // B format: bf16
-           | (static_cast<uint32_t>(a_mn) << 15)   // A major
-           | (static_cast<uint32_t>(b_mn) << 16)   // B major
-           | (static_cast<uint32_t>(N >> 3) << 17) // N / 8
-           | (static_cast<uint32_t>(M >> 4) << 24);// M / 16
+// in_f16: 1 when A and B are fp16 (format 0), 0 when they are bf16 (format 1).
+__host__ __device__ constexpr uint32_t idesc_f16_kind(int M, int N, int a_mn, int b_mn, int in_f16) {
+    return (1u << 4)                                    // D format: f32
+           | ((in_f16 ? 0u : 1u) << 7)                  // A format: f16 (0) / bf16 (1)
+           | ((in_f16 ? 0u : 1u) << 10)                 // B format: same type as A
+           | (static_cast<uint32_t>(a_mn) << 15)        // A major
+           | (static_cast<uint32_t>(b_mn) << 16)        // B major
+           | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }
 
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Exact widening of an fp16 bit pattern to fp32.
+__device__ __forceinline__ float f16_to_f32(uint16_t h) {
+    float r;
+    asm("cvt.f32.f16 %0, %1;" : "=f"(r) : "h"(h));
     return r;
 }
 
@@ -336,6 +376,15 @@ __device__ __forceinline__ uint32_t ld_shared_volatile_u32(uint32_t addr) {
 
 __device__ __forceinline__ void st_shared_volatile_u32(uint32_t addr, uint32_t v) {
     asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// 16-byte load from the shared memory of any CTA of the cluster (cluster address from mapa):
+// distributed shared memory.
+__device__ __forceinline__ void ld_cluster_v4(uint32_t addr_cluster, uint32_t& a, uint32_t& b, uint32_t& c,
+                                              uint32_t& d) {
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+                 : "r"(addr_cluster)
+                 : "memory");
 }
 
 // Store a word into the shared memory of a CTA of the cluster (cluster address).

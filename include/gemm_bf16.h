@@ -53,8 +53,10 @@ typedef enum {
 } gemm_status_t;
 
 typedef enum {
-    GEMM_OUT_F32 = 0, /* C is float32 */
-    GEMM_OUT_BF16 = 1 /* C is bfloat16 (fp32 result rounded to nearest even once) */
+    GEMM_OUT_F32 = 0,  /* C is float32 */
+    GEMM_OUT_BF16 = 1, /* C is bfloat16 (fp32 result rounded to nearest even once) */
+    GEMM_OUT_F16 = 2   /* C is IEEE binary16 (fp32 result rounded to nearest even once; values
+                          beyond +-65504 become +-inf) */
 } gemm_out_t;
 
 /*
@@ -101,14 +103,62 @@ GEMM_API gemm_status_t gemm_bf16_batched_shared_w(int batch, int M, int N, int K
                                          int ldy, long long stride_y, gemm_out_t out_type,
                                          float alpha, float beta, struct CUstream_st* stream);
 
+/*
+ * gemm_f16, gemm_f16_batched_shared_w -- the same operations, arguments, layouts, conventions
+ * and errors as gemm_bf16 and gemm_bf16_batched_shared_w, with A and B (W and X) holding IEEE
+ * binary16 (fp16) values instead of bfloat16.  Products are exact and accumulate in fp32, as
+ * for bf16.  The pages' GEMM measurements (page "Triton 3.7 permite extender el compilador de
+ * GPU sin forks", sections "NVIDIA H100 (Hopper): resultados de rendimiento" and "AMD MI350:
+ * GEMM segmentado") are FP16 GEMMs; this is that operand type.  The output may be fp32, bf16
+ * or fp16 (out_type).
+ */
+GEMM_API gemm_status_t gemm_f16(int M, int N, int K, const void* A, int lda, const void* B, int ldb,
+                                void* C, int ldc, gemm_out_t out_type, float alpha, float beta,
+                                struct CUstream_st* stream);
+
+GEMM_API gemm_status_t gemm_f16_batched_shared_w(int batch, int M, int N, int K, const void* W, int ldw,
+                                                 const void* X, int ldx, long long stride_x, void* Y,
+                                                 int ldy, long long stride_y, gemm_out_t out_type,
+                                                 float alpha, float beta, struct CUstream_st* stream);
+
+/*
+ * gemm_bf16_batched_shared_w_dedup -- Y[b] = alpha * W * X[index[b]] + beta * Y[b], b < batch:
+ * the shared-W form for requests whose items repeat feature entries.
+ *
+ * The recommendation-model kernel on the page "Meta accelere un noyau GPU d'un facteur 4 avec
+ * TLX, une extension du langage Triton" gets part of its speed-up from no longer handling
+ * repeated features as copies (sections "Comment le chargement des donnees gene le calcul":
+ * a buyer's data are identical across the items scored for that buyer; "Ce que signifie une
+ * acceleration d'un facteur quatre").  Here the request carries each distinct entry once: X
+ * holds n_unique entries, X[u] = X + u*stride_x (K x N row-major, ldx >= max(1, N)), and
+ * item b uses entry index[b].  The GEMM runs once per distinct entry; its epilogue writes
+ * the result to every item that uses it (Y[b] = Y + b*stride_y, M x N row-major; when
+ * batch > 1, stride_y >= (M-1)*ldy + N).  The items of one entry receive bitwise the same
+ * values as gemm_bf16_batched_shared_w gives for the expanded batch X[b] = X[index[b]] when
+ * both calls take the same tile plan (no split of K is used here).
+ *
+ *   index  device memory, `batch` ints in [0, n_unique), 4-byte aligned; read by the device.
+ *          An entry outside that range leaves its item's Y untouched and makes the next
+ *          gemm_bf16_device_status return GEMM_ERR_INVALID_ARG.
+ * Other arguments, conventions and errors as gemm_bf16_batched_shared_w; n_unique < 0, or
+ * n_unique == 0 with work to do, or a NULL index with batch > 0 is GEMM_ERR_INVALID_ARG.  The
+ * workspace also holds the per-entry item lists (2*n_unique + 1 + batch ints).
+ */
+GEMM_API gemm_status_t gemm_bf16_batched_shared_w_dedup(int batch, int n_unique, int M, int N, int K,
+                                                        const void* W, int ldw, const void* X, int ldx,
+                                                        long long stride_x, const int* index, void* Y,
+                                                        int ldy, long long stride_y, gemm_out_t out_type,
+                                                        float alpha, float beta, struct CUstream_st* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 GEMM_API const char* gemm_bf16_status_string(gemm_status_t s);
 
 /*
  * gemm_bf16_device_status -- synchronizes `stream`, then reports whether any kernel of this
  * library that ran on the current device since the previous call gave up a bounded
- * barrier wait (GEMM_ERR_TIMEOUT; the word is then cleared), or GEMM_ERR_CUDA if the
- * synchronization failed, else GEMM_OK.  A timed-out kernel skips its remaining tiles,
+ * barrier wait (GEMM_ERR_TIMEOUT), or found a deduplicated batch's index out of range
+ * (GEMM_ERR_INVALID_ARG); the word is then cleared.  GEMM_ERR_CUDA if the synchronization
+ * failed, else GEMM_OK.  A timed-out kernel skips its remaining tiles,
  * releases its tensor memory and exits, so the CUDA context stays usable; its output is
  * incomplete.
  */
@@ -129,13 +179,20 @@ GEMM_API gemm_status_t gemm_bf16_device_status(struct CUstream_st* stream);
  * Returns GEMM_ERR_INVALID_ARG for an unknown plan.  A plan that cannot serve a given
  * call is replaced by the automatic choice for that call.
  *
- * With few output tiles and a long K, plans 0-4 and 8 may also cut K into slices (split-K): each
- * (tile, slice) unit writes fp32 partial sums to the workspace and the last unit of a tile
- * adds them in slice order, so results stay bitwise reproducible.  The plan and the slice
- * count come from a cost model; environment variables read at every call override it for
+ * With few output tiles and a long K, the kernels may also cut K into slices, in one of two ways:
+ *   cluster split-K (plans 0, 1 and 8): the 2, 4 or 8 slices of a tile run on the CTAs of one
+ *     thread-block cluster, which add their partial tiles through distributed shared memory
+ *     (no workspace, so gemm_bf16_noalloc may use it too);
+ *   split-K through the workspace (plans 0-4 and 8): each (tile, slice) unit writes fp32
+ *     partial sums to the workspace and the last unit of a tile adds them.
+ * Both add the slices in slice order, so results stay bitwise reproducible.  The plan and the
+ * slice count come from a cost model; environment variables read at every call override it for
  * sweeps and tests:
- *   GEMM_BF16_SPLIT_K=s     (1..8) s slices wherever the plan and K allow it (1: never split)
- *   GEMM_BF16_GROUP_M=g     (1..64) m-blocks per group of the persistent tile order
+ *   GEMM_BF16_SPLIT_K=s        (1..8) s workspace slices wherever the plan and K allow it
+ *                              (1: no split of either kind unless the next variable forces one)
+ *   GEMM_BF16_CLUSTER_SPLIT=s  (2, 4, 8) cluster split-K with s slices where the plan takes it;
+ *                              1: never cluster split-K
+ *   GEMM_BF16_GROUP_M=g        (1..64) m-blocks per group of the persistent tile order
  */
 GEMM_API gemm_status_t gemm_bf16_set_plan(int plan);
 
@@ -180,6 +237,72 @@ GEMM_API gemm_status_t gemm_bf16_set_wait_timeout_ns(unsigned long long ns);
 GEMM_API gemm_status_t gemm_bf16_noalloc(int M, int N, int K, const void* A, int lda, const void* B,
                                          int ldb, void* C, int ldc, gemm_out_t out_type,
                                          float alpha, float beta, struct CUstream_st* stream);
+
+/*
+ * gemm_bf16_tensor_map_cache_stats -- how many tensor maps (the TMA descriptors of A, B and C)
+ * the calls so far took from the library's cache (*hits) and had to encode (*misses).  A map
+ * depends only on a buffer's address, extents, strides and tile box, so repeated calls on the
+ * same buffers encode nothing.  GEMM_ERR_INVALID_ARG if a pointer is NULL.
+ */
+GEMM_API gemm_status_t gemm_bf16_tensor_map_cache_stats(unsigned long long* hits,
+                                                        unsigned long long* misses);
+
+/*
+ * Autotuning.  The pages integrate TLX with Triton's autotuning (page "Meta presente TLX pour
+ * combler le fosse...", section "Comment cela fonctionne"); here the tuner searches this
+ * library's own configuration space for one problem: the tile plan (0-8 above), K cut into 2, 4
+ * or 8 slices through the workspace or across a cluster of 2, 4 or 8 CTAs (few-tile problems),
+ * and the raster group of the persistent tile order (4, 8 or 16 m-blocks; many-tile problems).
+ *
+ * gemm_autotune -- times every candidate configuration on the given operands and records the
+ * fastest in a per-process table.  Later calls of the same problem -- same device SM count,
+ * form, sizes, operand and output types, beta == 0 or not, and the same alignment of A, B and C
+ * (which decides the pre-pass and store paths) -- take the recorded configuration instead of
+ * the library's cost model, unless a plan or split is forced (gemm_bf16_set_plan, the
+ * GEMM_BF16_* variables).
+ *
+ *   in_type  0: bf16 operands, 1: fp16 operands.
+ *   form     0: gemm_bf16 / gemm_f16 (batch must be 1; stride_b, stride_c, index and n_unique
+ *               are ignored); 1: the batched shared-W form (B = X N-major, stride_b = stride_x,
+ *               stride_c = stride_y); 2: the deduplicated shared-W form (bf16 only; index and
+ *               n_unique as in gemm_bf16_batched_shared_w_dedup).
+ *   Other arguments as in the matching entry point.  C is NOT written: candidates write into
+ *   a scratch copy of C taken from the library's workspace pool.  *best_us (if best_us != NULL)
+ *   receives the winner's time per call in microseconds.
+ * Synchronous: returns after the measurements (it synchronizes `stream`); do not call it
+ * during stream capture.  Returns GEMM_OK, or an argument/CUDA error; GEMM_OK with nothing
+ * recorded when there is nothing to compute (an empty problem, K == 0 or alpha == 0).
+ */
+GEMM_API gemm_status_t gemm_autotune(int in_type, int form, int batch, int n_unique, int M, int N, int K,
+                                     const void* A, int lda, const void* B, int ldb, long long stride_b,
+                                     const int* index, const void* C, int ldc, long long stride_c,
+                                     gemm_out_t out_type, float alpha, float beta, struct CUstream_st* stream,
+                                     float* best_us);
+
+/* Empties the tuning table. */
+GEMM_API gemm_status_t gemm_tuning_clear(void);
+
+/* Number of problems in the tuning table. */
+GEMM_API int gemm_tuning_size(void);
+
+/*
+ * gemm_tuning_save / gemm_tuning_load -- write the tuning table to a text file, or add a file's
+ * entries to it (same key: replaced).  One line per problem:
+ *   gemmtune1 sms batch M N K n_unique b_mn in_f16 out c_read a_ok b_ok c_tma plan splits csplit group_m us
+ * (b_mn: batched forms; c_read: beta != 0; a_ok/b_ok: operand read in place by TMA; c_tma: C
+ * stored by TMA; splits: workspace K slices; csplit: cluster K slices; us: measured time).
+ * Lines starting with '#' and empty lines are skipped.  A file that cannot be opened, or any
+ * malformed line or impossible configuration, returns GEMM_ERR_INVALID_ARG and loads nothing.
+ */
+GEMM_API gemm_status_t gemm_tuning_save(const char* path);
+GEMM_API gemm_status_t gemm_tuning_load(const char* path);
+
+/*
+ * gemm_last_config -- the configuration of the calling thread's most recent GEMM kernel launch
+ * (plan, workspace K slices, cluster K slices, raster group); plan -1 before any launch.
+ * GEMM_ERR_INVALID_ARG if a pointer is NULL.
+ */
+GEMM_API gemm_status_t gemm_last_config(int* plan, int* splits, int* csplit, int* group_m);
 
 /* Library version as an integer (major*10000 + minor*100 + patch). */
 GEMM_API int gemm_bf16_version(void);

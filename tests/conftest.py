@@ -8,6 +8,17 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def build_library() -> str:
+    """Build libgemm_bf16.so if it is missing or stale and return its path.  _build.py is loaded
+    by path: importing the package itself would first load the (possibly stale) library."""
+    import importlib.util
+    path = os.path.join(ROOT, "dsl_persistent_warp_b200", "_build.py")
+    spec = importlib.util.spec_from_file_location("_pw_build_for_tests", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 

@@ -14,20 +14,21 @@ HEADER = os.path.join(ROOT, "include", "gemm_bf16.h")
 def _declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"GEMM_API\s+[\w\s\*]+?\b(gemm_bf16\w*)\s*\(", src)))
+    return sorted(set(re.findall(r"GEMM_API\s+[\w\s\*]+?\b(gemm_\w+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
 def capi():
-    from dsl_persistent_warp_b200 import _build
-    _build.build()
+    from conftest import build_library
+    build_library()
     from dsl_persistent_warp_b200 import capi as c
     return c
 
 
 def test_header_declares_the_boundary():
     names = _declared_functions()
-    for required in ("gemm_bf16", "gemm_bf16_batched_shared_w", "gemm_bf16_status_string"):
+    for required in ("gemm_bf16", "gemm_bf16_batched_shared_w", "gemm_bf16_status_string",
+                     "gemm_f16", "gemm_f16_batched_shared_w"):
         assert required in names
 
 
@@ -59,7 +60,8 @@ BAD_GEMM_CALLS = [
     (4, 4, 8, 16, 7, 16, 8, 16, 4, 1, 1.0, 0.0),    # lda < K
     (4, 4, 8, 16, 8, 16, 7, 16, 4, 1, 1.0, 0.0),    # ldb < K
     (4, 4, 8, 16, 8, 16, 8, 16, 3, 1, 1.0, 0.0),    # ldc < N
-    (4, 4, 8, 16, 8, 16, 8, 16, 4, 2, 1.0, 0.0),    # unknown out_type
+    (4, 4, 8, 16, 8, 16, 8, 16, 4, 3, 1.0, 0.0),    # unknown out_type
+    (4, 4, 8, 16, 8, 16, 8, 17, 4, 2, 1.0, 0.0),    # fp16 C not 2-byte aligned
     (4, 4, 8, 16, 8, 16, 8, None, 4, 1, 1.0, 0.0),  # NULL C
     (4, 4, 8, None, 8, 16, 8, 16, 4, 1, 1.0, 0.0),  # NULL A with work to do
     (4, 4, 8, 16, 8, None, 8, 16, 4, 1, 1.0, 0.0),  # NULL B with work to do
@@ -69,8 +71,9 @@ BAD_GEMM_CALLS = [
 
 
 @pytest.mark.parametrize("args", BAD_GEMM_CALLS)
-def test_gemm_rejects_bad_arguments(capi, args):
-    assert capi.gemm_bf16(*args, None) == capi.GEMM_ERR_INVALID_ARG
+@pytest.mark.parametrize("entry", ["gemm_bf16", "gemm_f16", "gemm_bf16_noalloc"])
+def test_gemm_rejects_bad_arguments(capi, args, entry):
+    assert getattr(capi, entry)(*args, None) == capi.GEMM_ERR_INVALID_ARG
 
 
 def test_empty_problems_are_ok_without_a_device(capi):
@@ -91,8 +94,15 @@ BAD_BATCHED = [
 
 
 @pytest.mark.parametrize("args", BAD_BATCHED)
-def test_batched_rejects_bad_arguments(capi, args):
-    assert capi.gemm_bf16_batched_shared_w(*args, None) == capi.GEMM_ERR_INVALID_ARG
+@pytest.mark.parametrize("entry", ["gemm_bf16_batched_shared_w", "gemm_f16_batched_shared_w"])
+def test_batched_rejects_bad_arguments(capi, args, entry):
+    assert getattr(capi, entry)(*args, None) == capi.GEMM_ERR_INVALID_ARG
+
+
+def test_tensor_map_cache_stats_without_a_device(capi):
+    """No call has reached the encoder in a process without a GPU: the cache is empty."""
+    assert capi.gemm_bf16_tensor_map_cache_stats() == (0, 0)
+    assert capi.LIB.gemm_bf16_tensor_map_cache_stats(None, None) == capi.GEMM_ERR_INVALID_ARG
 
 
 def test_set_plan_and_timeout(capi):
@@ -105,7 +115,7 @@ def test_set_plan_and_timeout(capi):
 
 def test_library_links_no_torch():
     """The boundary is plain C: the shared library depends on no PyTorch library."""
-    from dsl_persistent_warp_b200 import _build
-    path = _build.build()
+    from conftest import build_library
+    path = build_library()
     out = subprocess.run(["ldd", path], capture_output=True, text=True).stdout
     assert "torch" not in out and "c10" not in out

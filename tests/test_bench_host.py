@@ -6,6 +6,7 @@ import json
 import os
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -41,9 +42,10 @@ def test_roofline_bound_follows_the_ridge():
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     for name, w in bench.WORKLOADS.items():
         _, batch, M, N, K, *_ = w
-        intensity = 2.0 * batch * M * N * K / bench.algorithmic_bytes(w)
+        intensity = bench.executed_flops(w) / bench.algorithmic_bytes(w)
         # square and LLM shapes and 4099^3 above the ridge; the thin edges and RecSys below
-        expect_tensor = name in ("square4096", "square8192", "llm_up", "llm_down", "edge4099")
+        expect_tensor = name in ("square4096", "square8192", "llm_up", "llm_down", "edge4099",
+                                 "square4096_f16", "square8192_f16")
         assert (intensity >= ridge) == expect_tensor, (name, intensity, ridge)
 
 
@@ -74,3 +76,30 @@ def test_default_workload_is_the_headline_config():
     assert bench.DEFAULT_WORKLOAD == "square8192"
     _, batch, M, N, K, out, alpha, beta, *_ = bench.WORKLOADS["square8192"]
     assert (batch, M, N, K, out, alpha, beta) == (1, 8192, 8192, 8192, "bf16", 1.0, 0.0)
+
+
+def test_l2_flush_rule():
+    """Workloads whose data are under twice the L2 cache are timed cold (flushed); the others
+    run back to back."""
+    flushed = sorted(n for n, w in bench.WORKLOADS.items() if bench.needs_flush(w))
+    assert flushed == ["edge127x8191", "edge4099", "edge8192x256", "recsys_dedup128", "recsys_dedup4",
+                       "square256", "square4096", "square4096_f16"]
+
+
+def test_fp16_workloads_use_fp16_operands():
+    for name in ("square8192_f16", "square4096_f16"):
+        w = bench.WORKLOADS[name]
+        assert w.in_dtype == "f16" and w.out == "f16"
+    assert all(w.in_dtype == "bf16" for n, w in bench.WORKLOADS.items() if not n.endswith("_f16"))
+
+
+def test_dedup_workloads():
+    w = bench.WORKLOADS["recsys_dedup128"]
+    idx = bench.dedup_index(w)
+    assert idx.shape == (2048,) and idx.min() == 0 and idx.max() == 15
+    assert np.all(np.bincount(idx) == 128)  # 16 requests of 128 items
+    assert np.all(np.bincount(bench.dedup_index(bench.WORKLOADS["recsys_dedup4"])) == 4)
+    # X is read once per distinct entry; Y is written per item; the index is read once
+    assert bench.algorithmic_bytes(w) == 256 * 512 * 2 + 16 * 512 * 128 * 2 + 2048 * 256 * 128 * 2 + 2048 * 4
+    assert bench.executed_flops(w) == 2.0 * 16 * 256 * 128 * 512
+    assert bench.launches_per_step(w) == 2

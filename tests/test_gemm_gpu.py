@@ -8,8 +8,9 @@ import pytest
 import torch
 
 import oracle
-from parity import bits_of, check, sample_rows, to_dev_bf16, values_f64
-from synth import bf16_bits_to_f64, f64_to_bf16_bits, matrix_bf16, seed_for
+from parity import bits_of, check, sample_rows, to_dev_bf16, to_dev_f16, values_f64
+from synth import (bf16_bits_to_f64, f16_bits_to_f64, f64_to_bf16_bits, f64_to_f16_bits, matrix_bf16,
+                   matrix_f16, seed_for)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,12 +31,13 @@ def _plan(pw, plan):
 GUARD_ROWS = 3
 
 
-def _run(pw, A, B, M, N, K, *, out=torch.bfloat16, alpha=1.0, beta=0.0, c0=None, ldc=None):
-    """A: (M, lda) uint16 bits, B: (N, ldb) bits.  C lives in a buffer with GUARD_ROWS extra NaN
-    rows after row M-1; returns (C device view, buffer rows 0..M-1); the guard rows are checked
-    to be untouched here."""
-    dA = to_dev_bf16(A)[:, :K]
-    dB = to_dev_bf16(B)[:, :K]
+def _run(pw, A, B, M, N, K, *, out=torch.bfloat16, alpha=1.0, beta=0.0, c0=None, ldc=None, f16=False):
+    """A: (M, lda) uint16 bits, B: (N, ldb) bits (bf16, or fp16 with ``f16``).  C lives in a
+    buffer with GUARD_ROWS extra NaN rows after row M-1; returns (C device view, buffer rows
+    0..M-1); the guard rows are checked to be untouched here."""
+    dev = to_dev_f16 if f16 else to_dev_bf16
+    dA = dev(A)[:, :K]
+    dB = dev(B)[:, :K]
     ldc = N if ldc is None else ldc
     full = torch.full((M + GUARD_ROWS, ldc), float("nan"), dtype=out, device="cuda")
     if c0 is not None:
@@ -252,6 +254,94 @@ def test_split_k_unaligned_c(pw, monkeypatch):
     assert rep["ok"], rep
 
 
+# ----------------------------------------------------------------------------- cluster split-K
+CSPLIT_PLANS = [0, 1, 8]  # one-CTA streaming plans: the ones whose kernels take it
+CSPLIT_CASES = [(300, 200, 1100, 2), (129, 257, 1500, 4), (1000, 136, 2000, 8), (256, 512, 1024, 4),
+                (127, 1000, 2048, 4)]
+
+
+@pytest.mark.parametrize("plan", CSPLIT_PLANS)
+@pytest.mark.parametrize("case", CSPLIT_CASES, ids=[f"{m}x{n}x{k}_c{s}" for m, n, k, s in CSPLIT_CASES])
+def test_cluster_split_k(pw, plan, case, monkeypatch):
+    """K slices of a tile on the CTAs of one cluster, partial tiles added through distributed
+    shared memory: same tolerance as the unsplit path, alpha/beta with C in place, ragged M, N
+    and K; a second call gives the same bits."""
+    M, N, K, S = case
+    monkeypatch.setenv("GEMM_BF16_CLUSTER_SPLIT", str(S))
+    _plan(pw, plan)
+    A = matrix_bf16(161, M, K)
+    B = matrix_bf16(162, N, K)
+    c0bits = matrix_bf16(163, M, N)
+    c0 = torch.from_numpy(bf16_bits_to_f64(c0bits)).to(torch.bfloat16)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16, alpha=0.5, beta=1.0, c0=c0)
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, c0=c0bits, alpha=0.5, beta=1.0)
+    rep = check(values_f64(C), Cref, R, out_bf16=True)
+    assert rep["ok"], rep
+    C2, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16, alpha=0.5, beta=1.0, c0=c0)
+    assert torch.equal(C, C2)
+
+
+@pytest.mark.parametrize("plan", CSPLIT_PLANS)
+@pytest.mark.parametrize("S", [2, 4, 8])
+def test_cluster_split_k_integer_bit_exact(pw, plan, S, monkeypatch):
+    """Small-integer inputs: the slice sums and their total are exact in fp32, so the result is
+    bit-exact against the oracle, in fp32 and in bf16."""
+    monkeypatch.setenv("GEMM_BF16_CLUSTER_SPLIT", str(S))
+    _plan(pw, plan)
+    rng = np.random.default_rng(700 + plan + S)
+    M, N, K = 384, 272, 2048
+    A = f64_to_bf16_bits(rng.integers(-3, 4, (M, K)).astype(np.float64))
+    B = f64_to_bf16_bits(rng.integers(-3, 4, (N, K)).astype(np.float64))
+    Cref, _ = oracle.gemm(A, B, M=M, N=N, K=K)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.float32)
+    assert np.array_equal(values_f64(C), Cref)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16)
+    assert np.array_equal(bits_of(C), f64_to_bf16_bits(Cref))
+
+
+def test_cluster_split_k_unaligned_c_and_fp16(pw, monkeypatch):
+    """Cluster split-K with an odd ldc (row-by-row epilogue) and packed lda/ldb (pre-pass), and
+    with fp16 operands and fp16 output."""
+    monkeypatch.setenv("GEMM_BF16_CLUSTER_SPLIT", "4")
+    _plan(pw, -1)
+    M, N, K = 127, 8191, 2048
+    A = matrix_bf16(171, M, K, ld=K)
+    B = matrix_bf16(172, N, K, ld=K)
+    c0bits = matrix_bf16(173, M, N, ld=N)
+    c0 = torch.from_numpy(bf16_bits_to_f64(c0bits)).to(torch.bfloat16)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16, alpha=0.5, beta=1.0, c0=c0, ldc=N)
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, c0=c0bits, alpha=0.5, beta=1.0)
+    rep = check(values_f64(C), Cref, R, out_bf16=True)
+    assert rep["ok"], rep
+    M, N, K = 300, 520, 3000
+    A = matrix_f16(174, M, K)
+    B = matrix_f16(175, N, K)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.float16, f16=True)
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, in_dtype="f16")
+    rep = check(values_f64(C), Cref, R, out_bf16=False, out_f16=True)
+    assert rep["ok"], rep
+
+
+@pytest.mark.parametrize("plan", CSPLIT_PLANS)
+def test_batched_cluster_split_k(pw, plan, monkeypatch):
+    """Cluster split-K on the batched shared-W call (MN-major X)."""
+    monkeypatch.setenv("GEMM_BF16_CLUSTER_SPLIT", "2")
+    _plan(pw, plan)
+    batch, M, N, K = 3, 200, 128, 2048
+    W = matrix_bf16(181, M, K, std=K ** -0.5)
+    X = matrix_bf16(182, batch * K, N)
+    y0 = torch.randn(batch, M, N, dtype=torch.float32).to(torch.bfloat16)
+    Y = y0.clone().cuda()
+    pw.gemm_bf16_batched_shared_w(to_dev_bf16(W), to_dev_bf16(X).view(batch, K, N), Y, alpha=0.5, beta=1.0)
+    torch.cuda.synchronize()
+    assert pw.device_status() == 0
+    Cref, R = oracle.gemm_batched(W, X, batch=batch, M=M, N=N, K=K, stride_x=K * N,
+                                  y0=y0.to(torch.float32).numpy().reshape(batch * M, N), stride_y=M * N,
+                                  alpha=0.5, beta=1.0)
+    rep = check(values_f64(Y), Cref, R, out_bf16=True)
+    assert rep["ok"], rep
+
+
 def test_abi_errors_on_gpu(pw):
     c = pw.capi
     t = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
@@ -356,7 +446,7 @@ def test_llm_mlp_shapes(pw, which):
     """LLM MLP GEMMs: up-proj 16384x28672x8192 and down-proj 16384x8192x28672, activations
     N(0,1), weights N(0,0.02), bf16 out: sampled rows vs the oracle."""
     M, N, K = (16384, 28672, 8192) if which == "up" else (16384, 8192, 28672)
-    _full_case(pw, 2, M, N, K, std_b=0.02, rows=sample_rows(M, seed=K, per_block=1))
+    _full_case(pw, 2, M, N, K, std_b=0.02, rows=sample_rows(M, seed=K))
 
 
 EDGE = [(4099, 4099, 4099), (8192, 256, 4096), (127, 8191, 2048)]
@@ -408,3 +498,137 @@ def test_recsys_batched_config(pw):
         Cb, Rb = oracle.gemm(W, X[b * K:(b + 1) * K], M=M, N=N, K=K, b_kmajor=False)
         rep = check(values_f64(Y[int(b)]), Cb, Rb, out_bf16=True)
         assert rep["ok"], (int(b), rep)
+
+
+# ----------------------------------------------------------------------------- bit-exact at size
+def test_edge4099_integer_bit_exact(pw):
+    """M = N = K = 4099 with packed leading dimensions (alignment pre-pass for A and B, the
+    row-by-row epilogue for C), alpha = 0.5, beta = 1, small-integer A, B and C: every partial
+    sum and alpha*acc + beta*c0 are exact in fp32, so the fp32 output equals the oracle bit for
+    bit and the bf16 output is its single round-to-nearest-even."""
+    _plan(pw, -1)
+    n = 4099
+    rng = np.random.default_rng(4099)
+    A = f64_to_bf16_bits(rng.integers(-2, 3, (n, n)).astype(np.float64))
+    B = f64_to_bf16_bits(rng.integers(-2, 3, (n, n)).astype(np.float64))
+    c0i = rng.integers(-2, 3, (n, n)).astype(np.float64)
+    Cref, _ = oracle.gemm(A, B, M=n, N=n, K=n, c0=c0i.astype(np.float32), alpha=0.5, beta=1.0)
+    C, _ = _run(pw, A, B, n, n, n, out=torch.float32, alpha=0.5, beta=1.0,
+                c0=torch.from_numpy(c0i.astype(np.float32)))
+    assert np.array_equal(values_f64(C), Cref)
+    C, _ = _run(pw, A, B, n, n, n, out=torch.bfloat16, alpha=0.5, beta=1.0,
+                c0=torch.from_numpy(c0i).to(torch.bfloat16))
+    assert np.array_equal(bits_of(C), f64_to_bf16_bits(Cref))
+
+
+BATCH_EXACT = [(6, 256, 128, 512), (3, 200, 264, 320)]
+
+
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("case", BATCH_EXACT, ids=[f"b{b}_{m}x{n}x{k}" for b, m, n, k in BATCH_EXACT])
+def test_batched_integer_bit_exact(pw, plan, case):
+    """Shared-W batches (MN-major X descriptors, packing for N = 128) with small-integer
+    inputs: bit-exact against the oracle in fp32 and in bf16."""
+    _plan(pw, plan)
+    batch, M, N, K = case
+    rng = np.random.default_rng(300 + plan)
+    W = f64_to_bf16_bits(rng.integers(-3, 4, (M, K)).astype(np.float64))
+    X = f64_to_bf16_bits(rng.integers(-3, 4, (batch * K, N)).astype(np.float64))
+    Cref, _ = oracle.gemm_batched(W, X, batch=batch, M=M, N=N, K=K, stride_x=K * N)
+    dW, dX = to_dev_bf16(W), to_dev_bf16(X).view(batch, K, N)
+    for out in (torch.float32, torch.bfloat16):
+        Y = pw.gemm_bf16_batched_shared_w(dW, dX, out_dtype=out)
+        torch.cuda.synchronize()
+        assert pw.device_status() == 0
+        if out == torch.float32:
+            assert np.array_equal(values_f64(Y), Cref)
+        else:
+            assert np.array_equal(bits_of(Y), f64_to_bf16_bits(Cref))
+
+
+# ----------------------------------------------------------------------------- fp16 operands
+@pytest.mark.parametrize("plan", PLANS)
+def test_f16_integer_bit_exact(pw, plan):
+    """fp16 operands: A holds integers up to +-1000 (exact in fp16, not in bf16), B holds
+    -1, 0, 1; every partial sum is an exact integer below 2^24, so the fp32 output equals the
+    oracle bit for bit, and an fp16 output is its single rounding."""
+    _plan(pw, plan)
+    rng = np.random.default_rng(500 + plan)
+    M, N, K = 512, 384, 704
+    A = f64_to_f16_bits(rng.integers(-1000, 1001, (M, K)).astype(np.float64))
+    B = f64_to_f16_bits(rng.integers(-1, 2, (N, K)).astype(np.float64))
+    Cref, _ = oracle.gemm(A, B, M=M, N=N, K=K, in_dtype="f16")
+    C, _ = _run(pw, A, B, M, N, K, out=torch.float32, f16=True)
+    assert np.array_equal(values_f64(C), Cref)
+    C, _ = _run(pw, A, B, M, N, K, out=torch.bfloat16, f16=True)
+    assert np.array_equal(bits_of(C), f64_to_bf16_bits(Cref))
+
+
+F16_SHAPES = [(129, 257, 65), (300, 200, 1100), (513, 264, 72), (1000, 16, 130)]
+
+
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("shape", F16_SHAPES, ids=[f"{m}x{n}x{k}" for m, n, k in F16_SHAPES])
+def test_f16_ragged(pw, plan, shape):
+    """fp16 operands (values down to the subnormal range) and every output type, with
+    alpha/beta and C read in place, ragged M, N and K."""
+    _plan(pw, plan)
+    M, N, K = shape
+    A = matrix_f16(111, M, K, std=0.05, ld=K + (8 - K % 8) % 8)
+    B = matrix_f16(112, N, K, ld=K + (8 - K % 8) % 8)
+    for out in (torch.float16, torch.float32, torch.bfloat16):
+        ldc = N + (8 - N % 8) % 8 + 8
+        c0 = torch.from_numpy(f16_bits_to_f64(matrix_f16(113, M, N, ld=ldc))).to(out)
+        C, buf = _run(pw, A, B, M, N, K, out=out, alpha=0.5, beta=1.0, c0=c0, ldc=ldc, f16=True)
+        c0_np = c0[:, :N].to(torch.float32).numpy()
+        Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, c0=c0_np, alpha=0.5, beta=1.0, in_dtype="f16")
+        rep = check(values_f64(C), Cref, R, out_bf16=out == torch.bfloat16, out_f16=out == torch.float16)
+        assert rep["ok"], (out, rep)
+        pad_before = c0[:, N:].to(torch.float32).numpy()
+        pad_after = buf[:, N:].cpu().to(torch.float32).numpy()
+        assert np.array_equal(np.isnan(pad_before), np.isnan(pad_after))
+
+
+@pytest.mark.parametrize("plan", PLANS)
+def test_f16_batched_shared_w(pw, plan):
+    _plan(pw, plan)
+    batch, M, N, K = 5, 256, 128, 512
+    W = matrix_f16(121, M, K, std=512 ** -0.5)
+    X = matrix_f16(122, batch * K, N)
+    dW, dX = to_dev_f16(W), to_dev_f16(X).view(batch, K, N)
+    for out in (torch.float16, torch.float32):
+        Y = pw.gemm_bf16_batched_shared_w(dW, dX, out_dtype=out)
+        torch.cuda.synchronize()
+        assert pw.device_status() == 0
+        Cref, R = oracle.gemm_batched(W, X, batch=batch, M=M, N=N, K=K, stride_x=K * N, in_dtype="f16")
+        rep = check(values_f64(Y), Cref, R, out_bf16=False, out_f16=out == torch.float16)
+        assert rep["ok"], (out, rep)
+
+
+def test_f16_square8192(pw):
+    """M = N = K = 8192 with fp16 operands N(0,1) and fp16 output: sampled rows vs the oracle."""
+    _plan(pw, -1)
+    n = 8192
+    A = matrix_f16(seed_for(1, "A"), n, n)
+    B = matrix_f16(seed_for(1, "B"), n, n)
+    C, _ = _run(pw, A, B, n, n, n, out=torch.float16, f16=True)
+    rows = sample_rows(n, seed=16)
+    Cref, R = oracle.gemm(A, B, M=n, N=n, K=n, rows=rows, in_dtype="f16")
+    rep = check(values_f64(C[torch.as_tensor(rows, device="cuda")]), Cref, R, out_bf16=False, out_f16=True)
+    assert rep["ok"], rep
+
+
+# ----------------------------------------------------------------------------- tensor-map cache
+def test_tensor_map_cache_hits_on_repeated_calls(pw):
+    """A second call on the same buffers encodes no tensor map: its three maps (A, B, C) come
+    from the cache."""
+    _plan(pw, -1)
+    A = to_dev_bf16(matrix_bf16(131, 384, 256))
+    B = to_dev_bf16(matrix_bf16(132, 320, 256))
+    C = torch.empty((384, 320), dtype=torch.bfloat16, device="cuda")
+    pw.gemm_bf16(A, B, C)
+    h0, m0 = pw.capi.gemm_bf16_tensor_map_cache_stats()
+    pw.gemm_bf16(A, B, C)
+    torch.cuda.synchronize()
+    h1, m1 = pw.capi.gemm_bf16_tensor_map_cache_stats()
+    assert (h1 - h0, m1 - m0) == (3, 0)
