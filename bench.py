@@ -320,6 +320,63 @@ def time_steps(torch, run_step, steps, stream, flush_buf=None):
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
 
 
+def timed_region(torch, step, args, stream, flush, world, local):
+    """The K timed steps.  The step is captured into a CUDA graph (eagerly if capture fails) and
+    launched twice untimed (a graph holding workspace allocations maps them on first launch).
+    Back-to-back workloads (no flush): the K steps are one replay of a graph of K steps between
+    two events, so consecutive GEMMs start without a launch gap; each step's own time (median,
+    min) comes from a second pass of single-step replays.  Flushed workloads: each step is timed
+    on its own after the flush.  NVML clocks are sampled over the timed region.
+    Returns (timed_ms, per-step ms, clocks, single-step graph or None, graph used)."""
+    graph = None
+    if not args.eager:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step()
+            torch.cuda.synchronize()
+            for _ in range(2):
+                graph.replay()
+            torch.cuda.synchronize()
+        except Exception:
+            graph = None
+            torch.cuda.synchronize()
+    run = graph.replay if graph is not None else step
+    graph_k = None
+    if flush is None and graph is not None:
+        try:
+            graph_k = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_k):
+                for _ in range(args.steps):
+                    step()
+            torch.cuda.synchronize()
+            graph_k.replay()
+            torch.cuda.synchronize()
+        except Exception:
+            graph_k = None
+            torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    if graph_k is not None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        graph_k.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        timed_ms = e0.elapsed_time(e1)
+    else:
+        step_ms = time_steps(torch, run, args.steps, stream, flush)
+        timed_ms = sum(step_ms)
+    barrier(world)
+    clocks = sampler.stop()
+    if graph_k is not None:
+        step_ms = time_steps(torch, run, args.steps, stream, flush)
+    del graph_k
+    return timed_ms, step_ms, clocks, graph, graph is not None
+
+
 def run_ours(args, w, wname):
     import torch
     import dsl_persistent_warp_b200 as pw
@@ -346,46 +403,36 @@ def run_ours(args, w, wname):
         raise RuntimeError("kernel reported a bounded-wait timeout during warm-up")
 
     # Host cost of one call through the public API (Python wrapper, C ABI, planning, cached
-    # tensor maps, launch), measured on eager calls that the device runs back to back.
+    # tensor maps, launch), measured on eager calls that the device runs back to back; and of
+    # the C entry point alone (pointers prepared once, one ctypes call per GEMM).
     n_host = max(3, min(args.steps, 20))
     t0 = time.perf_counter()
     for _ in range(n_host):
         step()
     host_us = (time.perf_counter() - t0) * 1e6 / n_host
     torch.cuda.synchronize()
+    host_c_us = None
+    if batch == 1:
+        c = pw.capi
+        a = (M, N, K, dA.data_ptr(), K, dB.data_ptr(), K, dC.data_ptr(), N,
+             {"f32": c.GEMM_OUT_F32, "bf16": c.GEMM_OUT_BF16, "f16": c.GEMM_OUT_F16}[out], alpha, beta,
+             stream.cuda_stream)
+        fn = c.LIB.gemm_f16 if w.in_dtype == "f16" else c.LIB.gemm_bf16
+        t0 = time.perf_counter()
+        for _ in range(n_host):
+            fn(*a)
+        host_c_us = (time.perf_counter() - t0) * 1e6 / n_host
+        torch.cuda.synchronize()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if needs_flush(w) else None
     eager_ms = time_steps(torch, step, n_host, stream, flush)
 
-    # The step captured once into a CUDA graph and replayed: the device time of small GEMMs is
-    # not hidden behind Python call overhead.  If capture is not possible the steps run eagerly.
-    graph = None
-    if not args.eager:
-        try:
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                step()
-            torch.cuda.synchronize()
-            # Untimed launches first: a graph that holds the library's workspace allocations maps
-            # their memory on its first launch.
-            for _ in range(2):
-                graph.replay()
-            torch.cuda.synchronize()
-        except Exception:
-            graph = None
-            torch.cuda.synchronize()
-    run = graph.replay if graph is not None else step
-    sampler = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize()
-    sampler.start()
-    step_ms = time_steps(torch, run, args.steps, stream, flush)
-    barrier(world)
-    clocks = sampler.stop()
+    timed_ms, step_ms, clocks, graph, used_graph = timed_region(torch, step, args, stream, flush, world, local)
     if pw.device_status() != 0:
         raise RuntimeError("kernel reported a bounded-wait timeout in the timed region")
-    total_ms = max_over_ranks(sum(step_ms), world)
+    total_ms = max_over_ranks(timed_ms, world)
     value = aggregate_tflops(flops, args.steps, world, total_ms)
-    avg_launch_ms = sum(step_ms) / args.steps
+    avg_launch_ms = timed_ms / args.steps
+    run = graph.replay if graph is not None else step
 
     # Sustained leg: the same step back to back for a few seconds, so that the part reaches its
     # power-capped steady state; compared with the measured sustained peak.
@@ -407,6 +454,7 @@ def run_ours(args, w, wname):
                      "seconds": round(sus_ms * 1e-3, 3), "clocks": sus_clocks,
                      "l2": "back to back, no flush"}
     used_graph = graph is not None
+    flushed = flush is not None
     del graph
 
     # End to end through the public API with host buffers: every step copies its inputs from
@@ -493,7 +541,6 @@ def run_ours(args, w, wname):
         achieved, peak, r_unit = executed_flops(w) / (avg_launch_ms * 1e-3) / 1e12, peak_t, "TFLOP/s"
         peak_desc = f"{w.in_dtype} dense, burst ({peak_kind}; the bf16 figure: same tensor rate)"
     traffic = recorded_traffic(wname)
-    flushed = flush is not None
     res = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -521,8 +568,10 @@ def run_ours(args, w, wname):
                 "expanded batch; the distinct entries' GEMMs do batch/n_unique times fewer"}
                if w.n_unique else {}),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "timing": ("cuda-graph replay of one step, events around each replay"
-                       if used_graph else "eager, events around each step"),
+            "timing": ("value: one replay of a graph of the K steps between two events; "
+                       "median/min: single-step replays" if (used_graph and not flushed) else
+                       "cuda-graph replay of one step, events around each replay" if used_graph else
+                       "eager, events around each step"),
         },
         "pct_of_peak": {
             "of_measured_burst": round(100.0 * value / world / peak_t, 2),
@@ -541,7 +590,9 @@ def run_ours(args, w, wname):
         },
         "eager": {"ms_per_step": round(statistics.mean(eager_ms), 5),
                   "median_ms": round(statistics.median(eager_ms), 5),
-                  "host_us_per_call": round(host_us, 2), "calls": n_host},
+                  "host_us_per_call": round(host_us, 2),
+                  "host_us_per_call_c_abi": None if host_c_us is None else round(host_c_us, 2),
+                  "calls": n_host},
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
                 "pipeline": "2 buffer sets; upload, GEMM and download on separate streams"},
@@ -661,9 +712,8 @@ def run_reference(args, w, wname):
 
 def run_vendor(args, w, wname):
     """Vendor context: the same workload through torch.matmul / addmm (cuBLAS), timed with the
-    same protocol as ours (W eager warm-up steps, K steps captured in a CUDA graph, one untimed
-    launch of the graph, one timed replay).  Rank 0 only; not a target and not part of the
-    product path."""
+    same routine as ours (timed_region, L2 flush included).  Rank 0 only; not a target and not
+    part of the product path."""
     import torch
 
     rank = int(os.environ.get("RANK", "0"))
@@ -678,7 +728,6 @@ def run_vendor(args, w, wname):
         return
     torch.cuda.set_device(0)
     dA, dB, dC, host = make_inputs(w, torch)
-
     dI = torch.from_numpy(host["index"]).long().cuda() if w.n_unique else None
 
     def step():
@@ -697,28 +746,16 @@ def run_vendor(args, w, wname):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for _ in range(args.steps):
-            step()
-    torch.cuda.synchronize()
-    graph.replay()
-    torch.cuda.synchronize()
-    sampler = ClockSampler(0)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if needs_flush(w) else None
     stream = torch.cuda.current_stream()
-    sampler.start()
-    e0.record(stream)
-    graph.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
-    flops = 2.0 * batch * M * N * K
-    res = {**base, "value": round(flops * args.steps / (ms * 1e-3) / 1e12, 2), "n_gpus": 1,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
-           "higher_is_better": True, "dtype": w.in_dtype, "data": "synthetic", "clocks": clocks}
+    timed_ms, step_ms, clocks, graph, used_graph = timed_region(torch, step, args, stream, flush, 1, 0)
     del graph
+    flops = 2.0 * batch * M * N * K
+    res = {**base, "value": round(flops * args.steps / (timed_ms * 1e-3) / 1e12, 2), "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(timed_ms / args.steps, 5),
+           "median_ms": round(statistics.median(step_ms), 5), "min_ms": round(min(step_ms), 5),
+           "higher_is_better": True, "dtype": w.in_dtype, "data": "synthetic", "cold_l2": flush is not None,
+           "clocks": clocks}
     print(json.dumps(res), flush=True)
 
 

@@ -36,9 +36,6 @@
 #ifndef PW_OPERAND_L2_POLICY
 #define PW_OPERAND_L2_POLICY 1
 #endif
-#ifndef PW_SUBTILE_SKEW
-#define PW_SUBTILE_SKEW 1
-#endif
 
 namespace pw {
 
@@ -409,94 +406,6 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     umma_commit<2>(empty_r1 + 8u * st);
                 }
             };
-            if constexpr (NSUB == 2 && ARES == 0 && PW_SUBTILE_SKEW) {
-                // Two sub-tiles own both accumulator slots, so a tile's epilogue would hold up the
-                // next tile's first k-block.  Sub-tile 1 may instead trail sub-tile 0 by up to
-                // STAGES k-blocks, whose stages stay held until its MMAs are issued:
-                //  * in a unit's last STAGES-1 k-blocks sub-tile 1 waits, so sub-tile 0 -- and the
-                //    drain of slot 0 -- finish while sub-tile 1 completes the unit;
-                //  * at a unit's start, while slot 1 is still being drained, sub-tile 0 runs ahead.
-                // The queue of held stages lives in one register: per entry 8 bits -- stage (0-2),
-                // first k-block of its unit (3), last (4), in the unit's tail (5), unit tag (6-7).
-                static_assert(STAGES <= 8, "stage index in 3 bits");
-                uint64_t pq = 0;
-                int qn = 0;
-                auto mma_sub = [&](int sub, int st, bool first) {
-                    const uint32_t d_tmem = tmem_base + (uint32_t)(sub * BN);
-                    const uint64_t a_st = adesc0 + (uint64_t)((st * T::A_BYTES) >> 4);
-                    const uint64_t b_sub = bdesc0 + (uint64_t)((st * T::B_BYTES + sub * T::B_SUB_BYTES) >> 4);
-#pragma unroll
-                    for (int kk = 0; kk < T::BK / 16; ++kk)
-                        umma_f16<CG>(d_tmem, a_st + (uint64_t)((kk * 32) >> 4),
-                                     b_sub + (uint64_t)((B_MN ? kk * 2048 : kk * 32) >> 4), IDESC,
-                                     (!first || kk != 0) ? 1u : 0u);
-                };
-                // sub-tile 1 of the oldest held stage; false when a wait gave up
-                auto pop_sub1 = [&]() -> bool {
-                    const uint32_t e = (uint32_t)(pq & 0xFFu);
-                    if (e & 8u) {
-                        if (!wait_phase<CG, CG == 2>(bar_tempty(1), ((tph >> 1) & 1u) ^ 1u, slot_abort, rank,
-                                                     p.status, p.timeout_ns, kStatusMma))
-                            return false;
-                        tc_fence_after();
-                        tph ^= 2u;
-                    }
-                    mma_sub(1, (int)(e & 7u), (e & 8u) != 0u);
-                    if (e & 16u) commit_tfull(1);
-                    commit_empty((int)(e & 7u));
-                    pq >>= 8;
-                    --qn;
-                    return true;
-                };
-                uint32_t utag = 0;  // unit counter mod 4
-                for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters, utag = (utag + 1) & 3u) {
-                    int kb_lo, kb_hi;
-                    unit_k(u, kb_lo, kb_hi);
-                    // Slot 0's drain for this unit needs the epilogue past the unit before the
-                    // previous one: issue what is still held from those older units.
-                    while (ok && qn > 0 && (((utag - (uint32_t)(pq >> 6)) & 3u) >= 2u)) ok = pop_sub1();
-                    for (int kb = kb_lo; ok && kb < kb_hi; ++kb) {
-                        if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, rank, p.status, p.timeout_ns,
-                                                   kStatusMma)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        if (kb == kb_lo) {
-                            if (!wait_phase<CG, CG == 2>(bar_tempty(0), (tph & 1u) ^ 1u, slot_abort, rank, p.status,
-                                                         p.timeout_ns, kStatusMma)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            tph ^= 1u;
-                        }
-                        mma_sub(0, stage, kb == kb_lo);
-                        if (kb == kb_hi - 1) commit_tfull(0);
-                        const uint32_t e = (uint32_t)stage | (kb == kb_lo ? 8u : 0u) | (kb == kb_hi - 1 ? 16u : 0u) |
-                                           (kb >= kb_hi - (STAGES - 1) ? 32u : 0u) | (utag << 6);
-                        pq |= (uint64_t)e << (8 * qn);
-                        ++qn;
-                        while (ok && qn > 0) {
-                            if (qn < STAGES) {
-                                const uint32_t f = (uint32_t)(pq & 0xFFu);
-                                // slot 1 still being drained: let sub-tile 0 run ahead
-                                if ((f & 8u) && !(CG == 2 ? mbar_test_wait_cluster(bar_tempty(1), ((tph >> 1) & 1u) ^ 1u)
-                                                          : mbar_test_wait(bar_tempty(1), ((tph >> 1) & 1u) ^ 1u)))
-                                    break;
-                                // the unit's tail: hold sub-tile 1 back until sub-tile 0 has finished
-                                if ((f & 32u) && (f >> 6) == utag && kb < kb_hi - 1) break;
-                            }
-                            ok = pop_sub1();
-                        }
-                        if (++stage == STAGES) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
-                    }
-                }
-                while (ok && qn > 0) ok = pop_sub1();
-            } else {
             for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters) {
                 int kb_lo, kb_hi;
                 unit_k(u, kb_lo, kb_hi);
@@ -547,7 +456,6 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     tph ^= 3u;
                 }
             }
-            }
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -563,10 +471,28 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         bool ok = true;
         // alpha/beta, conversion and store of chunk c (STG_COLS columns) of sub-tile `sub` of the
         // tile (b, nb) for the 32-row slab starting at row0; v holds this lane's row.
+        // batch entry of chunk c of sub-tile `sub` of tile (b, nb) (several per tile when packed)
+        auto chunk_entry = [&](int b, int nb, int sub, int c) {
+            const int jc = c * T::STG_COLS;
+            const int tcol = sub * T::BN_CTA + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
+            return p.pack > 1 ? nb * p.pack + tcol / p.N : b;
+        };
+        // Does chunk c leave through one tensor store?  Yes when C is TMA-addressable up to the
+        // chunk's end (a ragged right edge or unaligned ldc takes the row-by-row path).
+        auto chunk_tma = [&](int b, int nb, int sub, int c) {
+            const int jc = c * T::STG_COLS;
+            const int tcol = sub * T::BN_CTA + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
+            const int colc = p.pack > 1 ? tcol % p.N : nb * T::TILE_N + tcol;
+            return p.c_tma && colc + T::STG_COLS <= p.n_store_tma && chunk_entry(b, nb, sub, c) < p.batch_real;
+        };
         // bout >= 0: store to output entry bout instead of the chunk's own batch entry (the
-        // deduplicated form's scatter; C_in is read from the same entry).
+        // deduplicated form's scatter; C_in is read from the same entry).  more != nullptr: the
+        // chunk also goes to entries more[0], more[step], ... (n_more of them); when it leaves
+        // through a tensor store and C is not read, those are extra tensor stores of the same
+        // staged chunk and the call returns true, else it returns false and stores only bout.
         auto finish_chunk = [&](int b, int nb, int row0, int row, int sub, int c, float (&v)[T::STG_COLS],
-                                int bout = -1) {
+                                int bout = -1, const int* more = nullptr, int n_more = 0, int step = 1) -> bool {
+            bool fanned = false;
             const int col_tile = sub * T::BN_CTA;  // column within the tile
             const int jc = c * T::STG_COLS;
             const int tcol = col_tile + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
@@ -581,7 +507,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             // A chunk goes out as one tensor store when C is TMA-addressable up to the
             // chunk's end; otherwise (unaligned ldc, a ragged right edge) the warp moves it
             // row by row through the staging buffer so that every access is coalesced.
-            const bool tma_chunk = p.c_tma && colc + T::STG_COLS <= p.n_store_tma && entry_in;
+            const bool tma_chunk = chunk_tma(b, nb, sub, c);
             const bool coop_chunk = !tma_chunk;
             const uint32_t sbuf = stg + buf * T::STG_BYTES;
             // the buffer may still be read by an earlier tensor store
@@ -722,7 +648,13 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     if (lane == 0) {
                         tma_store_3d(&tmC, sbuf, colc, row0, bb);
                         bulk_commit_group();
+                        if (!p.c_read)
+                            for (int k = 0; k < n_more; ++k) {
+                                tma_store_3d(&tmC, sbuf, colc, row0, __ldg(more + (size_t)k * step));
+                                bulk_commit_group();
+                            }
                     }
+                    fanned = !p.c_read;
                 } else {
                     // row by row: lane j writes element j (and j+32) of each row, coalesced.
                     // The column predicates and the swizzle-free part of the shared address are
@@ -763,6 +695,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 }
                 if (T::STG_BUFS == 2) buf ^= 1;
             }
+            return fanned;
         };
         // TMEM -> registers: chunk c (STG_COLS columns) of the slot whose lane-quarter row is trow.
         auto load_chunk = [&](uint32_t trow, int c, float (&v)[T::STG_COLS]) {
@@ -808,12 +741,6 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         // the staging-buffer image), piece (32-column block cb, lane quarter qq) at
         // ((cb * 4 + qq) << 12).
         const uint32_t xchg = sbase + T::OFF_A;
-        // batch entry of chunk c of sub-tile `sub` of tile (b, nb) (several per tile when packed)
-        auto chunk_entry = [&](int b, int nb, int sub, int c) {
-            const int jc = c * T::STG_COLS;
-            const int tcol = sub * T::BN_CTA + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
-            return p.pack > 1 ? nb * p.pack + tcol / p.N : b;
-        };
         for (int u = cluster_id; ok && u < p.tiles * UPT; u += num_clusters) {
             const int t = u / UPT;
             const int sl = u % UPT;  // split-K slice, or destination part of a deduplicated batch
@@ -883,12 +810,23 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                             __syncwarp();
                             if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * slot);
                         };
-                        if (k >= hi && ci == CPW - 1) release();
-                        for (bool first = true; k < hi; k += DS, first = false) {
-                            const int d = __ldg(p.dd_dst + k);
-                            if (!first) load_chunk(trow, c, v);
-                            if (ci == CPW - 1 && k + DS >= hi) release();
-                            finish_chunk(b, nb, row0, row, sub, c, v, d);
+                        if (k >= hi) {
+                            if (ci == CPW - 1) release();
+                        } else {
+                            // With C not read and the chunk leaving through a tensor store, it is
+                            // converted and staged once and every item gets a tensor store of it;
+                            // otherwise each item reloads the accumulator and is stored in turn.
+                            const bool fan = !p.c_read && chunk_tma(b, nb, sub, c);
+                            const int n_more = fan ? (hi - k - 1) / DS : 0;
+                            if (ci == CPW - 1 && (fan || k + DS >= hi)) release();
+                            finish_chunk(b, nb, row0, row, sub, c, v, __ldg(p.dd_dst + k), p.dd_dst + k + DS, n_more, DS);
+                            if (!fan) {
+                                for (k += DS; k < hi; k += DS) {
+                                    load_chunk(trow, c, v);
+                                    if (ci == CPW - 1 && k + DS >= hi) release();
+                                    finish_chunk(b, nb, row0, row, sub, c, v, __ldg(p.dd_dst + k));
+                                }
+                            }
                         }
                     } else {
                         // publish this slice's partial sums; the slot stays held for the fixup
