@@ -9,8 +9,8 @@ A step is one GEMM (one call: the persistent kernel, plus the alignment pre-pass
 an operand needs them) over the workload's synthetic inputs, already resident in HBM.
 Timing: W untimed warm-up steps; the step is captured into a CUDA graph, and each of the K
 timed steps is one replay between two CUDA events on the launching stream.  Workloads whose
-data are smaller than twice the L2 cache get a 256 MiB write between steps (L2 flushed: cold
-cache), outside the events; larger ones run back to back.  The K steps are bracketed by a
+data are smaller than twice the L2 cache get a 256 MiB write and a 256 MiB read between steps
+(L2 flushed: cold and clean), outside the events; larger ones run back to back.  The K steps are bracketed by a
 barrier and a device synchronize; the time is the max over ranks.  The line reports the mean
 (value, ms_per_step), median and minimum step time.  A separate sustained leg replays the
 step back to back for a few seconds (the part settles at its power cap) and is compared with
@@ -303,16 +303,31 @@ def needs_flush(w) -> bool:
     return algorithmic_bytes(w) < 2 * L2_BYTES
 
 
+class L2Flush:
+    """Empties L2 before a step: a write of a buffer larger than L2, then a read of a second one,
+    so the step starts with none of its data cached and no dirty line left over from the flush
+    for it to write back."""
+
+    def __init__(self, torch):
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+        self.acc = torch.empty((), dtype=torch.float32, device="cuda")
+
+    def __call__(self, i):
+        self.w.fill_(i & 0x7F)
+        self.acc.copy_(self.r.sum())
+
+
 def time_steps(torch, run_step, steps, stream, flush_buf=None):
     """Device time (ms) of each of `steps` calls of run_step, each between two CUDA events on
-    `stream`; with `flush_buf`, a write of that buffer (larger than L2) precedes every step,
-    outside the events.  The host enqueues ahead of the device, so no host latency falls
-    between a step's events."""
+    `stream`; with `flush_buf` (an L2Flush), L2 is flushed before every step, outside the
+    events.  The host enqueues ahead of the device, so no host latency falls between a step's
+    events."""
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     for i in range(steps):
         if flush_buf is not None:
-            flush_buf.fill_(i & 0x7F)
+            flush_buf(i)
         starts[i].record(stream)
         run_step()
         ends[i].record(stream)
@@ -396,11 +411,29 @@ def run_ours(args, w, wname):
             pw.gemm_bf16_batched_shared_w(A, B, C, alpha=alpha, beta=beta)
 
     stream = torch.cuda.current_stream()
+    tuned = None
+    if args.autotune:
+        # The library's autotuner measures its configuration space on these operands first;
+        # the timed calls then take the configuration it recorded.
+        c = pw.capi
+        out_t = {"f32": c.GEMM_OUT_F32, "bf16": c.GEMM_OUT_BF16, "f16": c.GEMM_OUT_F16}[out]
+        form = 0 if batch == 1 else 2 if w.n_unique else 1
+        st, best_us = c.gemm_autotune(1 if w.in_dtype == "f16" else 0, form, batch, w.n_unique, M, N, K,
+                                      dA.data_ptr(), K, dB.data_ptr(), K if batch == 1 else N,
+                                      0 if batch == 1 else K * N, dI.data_ptr() if dI is not None else None,
+                                      dC.data_ptr(), N, 0 if batch == 1 else M * N, out_t, alpha, beta,
+                                      stream.cuda_stream)
+        if st != c.GEMM_OK:
+            raise RuntimeError(f"gemm_autotune: {c.gemm_bf16_status_string(st)}")
+        step()
+        torch.cuda.synchronize()
+        tuned = dict(zip(("plan", "splits", "csplit", "group_m"), c.gemm_last_config()), tuner_us=round(best_us, 2))
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     if pw.device_status() != 0:
         raise RuntimeError("kernel reported a bounded-wait timeout during warm-up")
+    config_used = dict(zip(("plan", "splits", "csplit", "group_m"), pw.capi.gemm_last_config()))
 
     # Host cost of one call through the public API (Python wrapper, C ABI, planning, cached
     # tensor maps, launch), measured on eager calls that the device runs back to back; and of
@@ -423,7 +456,7 @@ def run_ours(args, w, wname):
             fn(*a)
         host_c_us = (time.perf_counter() - t0) * 1e6 / n_host
         torch.cuda.synchronize()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if needs_flush(w) else None
+    flush = L2Flush(torch) if needs_flush(w) else None
     eager_ms = time_steps(torch, step, n_host, stream, flush)
 
     timed_ms, step_ms, clocks, graph, used_graph = timed_region(torch, step, args, stream, flush, world, local)
@@ -561,13 +594,15 @@ def run_ours(args, w, wname):
             "name": wname,
             "batch": batch, "M": M, "N": N, "K": K,
             "in": w.in_dtype, "out": out, "alpha": alpha, "beta": beta,
-            "l2": "flushed before every step (256 MiB write, outside the events)" if flushed else
+            "l2": "flushed before every step (256 MiB write, then 256 MiB read; outside the events)" if flushed else
                   "inputs larger than L2 (steps back to back)",
             "cold_l2": flushed,
             **({"n_unique": w.n_unique, "flops": "counted per item (2*M*N*K per item), as for the "
                 "expanded batch; the distinct entries' GEMMs do batch/n_unique times fewer"}
                if w.n_unique else {}),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "kernel_config": config_used,
+            "autotuned": tuned,
             "timing": ("value: one replay of a graph of the K steps between two events; "
                        "median/min: single-step replays" if (used_graph and not flushed) else
                        "cuda-graph replay of one step, events around each replay" if used_graph else
@@ -746,7 +781,7 @@ def run_vendor(args, w, wname):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if needs_flush(w) else None
+    flush = L2Flush(torch) if needs_flush(w) else None
     stream = torch.cuda.current_stream()
     timed_ms, step_ms, clocks, graph, used_graph = timed_region(torch, step, args, stream, flush, 1, 0)
     del graph
@@ -774,6 +809,8 @@ def main():
                     help="CPU seconds for the whole --impl reference run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager calls instead of a graph replay")
+    ap.add_argument("--autotune", action="store_true",
+                    help="run the library's autotuner on the workload before timing it")
     ap.add_argument("--sustained-seconds", type=float, default=None,
                     help="length of the back-to-back sustained leg (default: 3 s for tensor-bound "
                          "workloads, 0 otherwise)")

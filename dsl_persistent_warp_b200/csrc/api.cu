@@ -344,7 +344,7 @@ constexpr int kSplitCountersPerCta = 4;
 // partial tiles are added through distributed shared memory.  Cost per tile beyond its slice's
 // mainloop: two cluster barriers and the partial-tile write (fixed), and each CTA's read of the
 // other slices' share of its part of the tile.
-constexpr double kClusterSplitFixedSec = 2e-6;
+constexpr double kClusterSplitFixedSec = 4e-6;
 constexpr double kClusterSplitBytesPerSec = 150e9;
 
 // Can plan `i` serve this request?
@@ -472,9 +472,14 @@ Choice choose(const Req& r, int sms, bool allow_split) {
             const PlanDesc& pd = kPlans[i];
             if (!plan_csplit_ok(pd)) continue;
             if (only >= 0 ? i != only : (pd.rate <= 0.0 || !plan_serves(i, r))) continue;
+            const long long tiles = plan_tiles(pd, r);
             for (int cs = 2; cs <= 8; cs *= 2) {
                 if (fcs > 0 && cs != fcs) continue;
                 if (!split_valid(pd, r, cs) || cdiv(r.K, pd.bk) < (long long)cs * 2) continue;
+                // Automatically only where the unsplit tiles leave at least half the SMs idle and
+                // the split tiles still fit in one wave: measured on B200, a split that adds a
+                // wave (8192x256x4096: 37.8 -> 50 us) or only fills the last SMs loses.
+                if (fcs == 0 && (2 * tiles > sms || tiles * cs > sms)) continue;
                 const double t = plan_time_csplit(i, r, sms, cs);
                 if (fcs > 0 || (t < cbar && t < best_t * 0.999)) {
                     best = {i, 1, cs};
@@ -489,6 +494,9 @@ Choice choose(const Req& r, int sms, bool allow_split) {
     for (int i = 0; i < kNumPlans; ++i) {
         const PlanDesc& pd = kPlans[i];
         if (only >= 0 ? i != only : (pd.rate <= 0.0 || !plan_serves(i, r))) continue;
+        // Only few-tile problems (at least half the clusters idle unsplit): with many tiles the
+        // partial sums' traffic swamps the gain (4096^3, plan 4, two slices: 102 -> 175 us).
+        if (2 * plan_tiles(pd, r) > sms / pd.cg) continue;
         long long smax = cdiv(r.K, pd.bk) / kMinSplitKBlocks;
         if (smax > kMaxSplits) smax = kMaxSplits;
         for (int sp = 2; sp <= (int)smax; ++sp) {

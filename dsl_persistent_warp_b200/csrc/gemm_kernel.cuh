@@ -36,6 +36,9 @@
 #ifndef PW_OPERAND_L2_POLICY
 #define PW_OPERAND_L2_POLICY 1
 #endif
+#ifndef PW_B_L2_POLICY
+#define PW_B_L2_POLICY PW_OPERAND_L2_POLICY
+#endif
 
 namespace pw {
 
@@ -295,15 +298,14 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint32_t full_leader0 = CG == 2 ? map_to_rank(bar_full(0), 0) : bar_full(0);
-            // A and B panels are read by several CTAs of a wave: keep them in L2 (build option
-            // PW_OPERAND_L2_POLICY: 0 evict-normal, 1 evict-last, 2 evict-first).
-#if PW_OPERAND_L2_POLICY == 0
-            const uint64_t pol = l2_policy_evict_normal();
-#elif PW_OPERAND_L2_POLICY == 2
-            const uint64_t pol = l2_policy_evict_first();
-#else
-            const uint64_t pol = l2_policy_evict_last();
-#endif
+            // A and B panels are read by several CTAs of a wave: keep them in L2 (build options
+            // PW_OPERAND_L2_POLICY for A and PW_B_L2_POLICY for B: 0 evict-normal, 1 evict-last,
+            // 2 evict-first).
+            auto policy = [](int k) {
+                return k == 0 ? l2_policy_evict_normal() : k == 2 ? l2_policy_evict_first() : l2_policy_evict_last();
+            };
+            const uint64_t pol = policy(PW_OPERAND_L2_POLICY);
+            const uint64_t pol_b = policy(PW_B_L2_POLICY);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = p.test_stall == 0;
@@ -344,8 +346,8 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     // This CTA's B chunk: tile columns [rank*B_CHUNK, +B_CHUNK), contiguous.
                     const int b_row = nb * T::TILE_N + (int)rank * T::B_CHUNK;
                     if constexpr (!B_MN) {
-                        if constexpr (CG == 1) tma_load_3d(sb, &tmB, full_bar, k0, b_row, b, pol);
-                        else tma_load_3d_pair(sb, &tmB, full_bar, k0, b_row, b, pol);
+                        if constexpr (CG == 1) tma_load_3d(sb, &tmB, full_bar, k0, b_row, b, pol_b);
+                        else tma_load_3d_pair(sb, &tmB, full_bar, k0, b_row, b, pol_b);
                     } else {
 #pragma unroll
                         for (int j = 0; j < T::B_CHUNK / 64; ++j) {
@@ -354,9 +356,9 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                             const int bx = p.pack > 1 ? nb * p.pack + tc / p.N : b;
                             const int cx = p.pack > 1 ? tc % p.N : b_row + 64 * j;
                             if constexpr (CG == 1)
-                                tma_load_3d(sb + j * T::MN_BOX_BYTES, &tmB, full_bar, cx, k0, bx, pol);
+                                tma_load_3d(sb + j * T::MN_BOX_BYTES, &tmB, full_bar, cx, k0, bx, pol_b);
                             else
-                                tma_load_3d_pair(sb + j * T::MN_BOX_BYTES, &tmB, full_bar, cx, k0, bx, pol);
+                                tma_load_3d_pair(sb + j * T::MN_BOX_BYTES, &tmB, full_bar, cx, k0, bx, pol_b);
                         }
                     }
                     if (++stage == STAGES) {

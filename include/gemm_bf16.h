@@ -222,7 +222,8 @@ GEMM_API gemm_status_t gemm_bf16_set_wait_timeout_ns(unsigned long long ns);
  * makes (needed when lda or ldb is not a multiple of 8 elements or a base is not 16-byte
  * aligned).  If those copies, each rounded up to 256 bytes, need more than the scratch holds,
  * the call returns GEMM_ERR_INVALID_ARG and enqueues nothing.  Calls whose operands need no
- * copy do not touch the scratch.
+ * copy do not touch the scratch.  K is never cut through the workspace here; the cluster form
+ * of split-K (partial sums exchanged in shared memory) needs no memory and may be used.
  *
  * The scratch is shared by every call on a device and keeps the last call's contents; nothing
  * in it has to start at zero (the copies are fully rewritten by each call that uses them, and
