@@ -253,7 +253,7 @@ GEMM_API gemm_status_t gemm_bf16_tensor_map_cache_stats(unsigned long long* hits
  * combler le fosse...", section "Comment cela fonctionne"); here the tuner searches this
  * library's own configuration space for one problem: the tile plan (0-8 above), K cut into 2, 4
  * or 8 slices through the workspace or across a cluster of 2, 4 or 8 CTAs (few-tile problems),
- * and the raster group of the persistent tile order (4, 8 or 16 m-blocks; many-tile problems).
+ * and the raster group of the persistent tile order (8, 16 or 32 m-blocks; many-tile problems).
  *
  * gemm_autotune -- times every candidate configuration on the given operands and records the
  * fastest in a per-process table.  Later calls of the same problem -- same device SM count,
