@@ -750,6 +750,27 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             decode_tile(p, t, b, mb, nb);
             const int row0 = mb * T::BM + (int)rank * 128 + 32 * q;
             const int row = row0 + (int)lane;
+            if (p.c_read && p.dd_off == nullptr && (S == 1 || sl == 0) && row < p.M && b < p.batch_real) {
+                // C_in of this warp's rows of the tile, fetched into L2 while the mainloop runs:
+                // the beta term then reads L2 instead of DRAM (a tile's epilogue is exposed when a
+                // CTA has a single tile).  Each lane asks for the first and last line of each of its
+                // row's chunk segments, within the matrix only (C rows may start anywhere).
+                constexpr int ES = OUT != OUT_F32 ? 2 : 4;
+#pragma unroll 1
+                for (int sub = 0; sub < NSUB; ++sub)
+#pragma unroll 1
+                    for (int ci = 0; ci < CPW; ++ci) {
+                        const int jc = (half * CPW + ci) * T::STG_COLS;
+                        const int tcol = sub * T::BN_CTA + (jc / T::BN_CTA) * T::B_CHUNK + jc % T::BN_CTA;
+                        const int bb = p.pack > 1 ? nb * p.pack + tcol / p.N : b;
+                        const int colc = p.pack > 1 ? tcol % p.N : nb * T::TILE_N + tcol;
+                        if (bb >= p.batch_real || colc >= p.N) continue;
+                        const char* seg = static_cast<const char*>(p.C) +
+                                          ((long long)bb * p.stride_c + (long long)row * p.ldc + colc) * ES;
+                        prefetch_l2(seg);
+                        prefetch_l2(seg + (min(T::STG_COLS, p.N - colc) * ES - 1));
+                    }
+            }
             // this warp's partials of slice s of the tile: pieces in (sub, ci, piece) order
             auto slab = [&](int s) { return p.ws + ((size_t)(t * CG + (int)rank) * S + s) * WS_TILE + (size_t)ew * WS_WARP; };
             if (S > 1) {

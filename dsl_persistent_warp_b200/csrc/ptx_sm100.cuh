@@ -366,6 +366,11 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr_cluster, uint32_t v
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr_cluster), "r"(v) : "memory");
 }
 
+// Hint: bring the 128-byte line holding `ptr` into L2 (no data returned).
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
 __device__ __forceinline__ void nanosleep_ns(uint32_t ns) {
     asm volatile("nanosleep.u32 %0;" ::"r"(ns));
 }
