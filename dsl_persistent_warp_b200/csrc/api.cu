@@ -441,7 +441,8 @@ int forced_csplit() {
 // Plan and K split for a request on a device with `sms` SMs (auto unless overridden); without
 // `allow_split` no global split-K (it needs workspace); cluster split-K needs none.
 Choice choose(const Req& r, int sms, bool allow_split) {
-    const int fs = allow_split ? forced_splits() : 1;
+    const int fs_env = forced_splits();  // GEMM_BF16_SPLIT_K (0: unset)
+    const int fs = allow_split ? fs_env : 1;
     const int fcs = r.index != nullptr ? 1 : forced_csplit();  // dedup units replace K slices
     const int forced = g_plan_override.load();
     int only = -1;  // the one plan to consider, or -1 for every streaming plan
@@ -469,7 +470,7 @@ Choice choose(const Req& r, int sms, bool allow_split) {
     }
     // Cluster split-K (no workspace): forced, or, when no split is forced either way, where it
     // beats the best so far by 10 %.
-    if (fcs > 1 || (fs == 0 && fcs == 0)) {
+    if (fcs > 1 || (fs_env == 0 && fcs == 0)) {
         const double cbar = best_t * 0.90;
         for (int i = 0; i < kNumPlans; ++i) {
             const PlanDesc& pd = kPlans[i];

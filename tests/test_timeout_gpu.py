@@ -22,13 +22,23 @@ pytestmark = pytest.mark.gpu
 def capi():
     from dsl_persistent_warp_b200 import capi as c
     yield c
-    os.environ.pop("GEMM_BF16_TEST_STALL_LOADS", None)
+    for k in ("GEMM_BF16_TEST_STALL_LOADS", "GEMM_BF16_CLUSTER_SPLIT", "GEMM_BF16_SPLIT_K"):
+        os.environ.pop(k, None)
     c.gemm_bf16_set_wait_timeout_ns(0)
     c.gemm_bf16_set_plan(-1)
 
 
-@pytest.mark.parametrize("plan", [0, 2, 4, 5])
-def test_expired_wait_reports_timeout_and_context_survives(capi, plan):
+# (plan, forced split): the persistent plans, and K cut across a cluster (every CTA of the cluster
+# must still reach both cluster barriers) or through the workspace.
+CASES = [(0, None), (2, None), (4, None), (5, None), (1, ("GEMM_BF16_CLUSTER_SPLIT", "2")),
+         (0, ("GEMM_BF16_CLUSTER_SPLIT", "4")), (0, ("GEMM_BF16_SPLIT_K", "2"))]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"plan{p}" + (f"_{e[0][10:]}{e[1]}" if e else "") for p, e in CASES])
+def test_expired_wait_reports_timeout_and_context_survives(capi, case):
+    plan, split = case
+    if split:
+        os.environ[split[0]] = split[1]
     import dsl_persistent_warp_b200 as pw
     M = N = K = 512
     A = matrix_bf16(71, M, K)

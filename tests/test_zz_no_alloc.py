@@ -77,6 +77,22 @@ def test_noalloc_takes_no_device_memory(capi):
     assert free1 == free0
 
 
+def test_noalloc_cuts_deep_k_across_a_cluster(capi):
+    """A few-tile, deep-K problem: the allocation-free entry point may still cut K, across the
+    CTAs of a cluster (partial sums exchanged in shared memory, no memory needed)."""
+    M, N, K = 512, 512, 8192
+    A, B = matrix_bf16(920, M, K, std=K ** -0.5), matrix_bf16(921, N, K)
+    dA, dB = to_dev_bf16(A), to_dev_bf16(B)
+    C = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    _call(capi.gemm_bf16_noalloc, capi, dA, K, dB, K, M, N, K, torch.float32, 1.0, 0.0, C)
+    torch.cuda.synchronize()
+    assert capi.gemm_bf16_device_status(_stream()) == 0
+    plan, splits, csplit, _ = capi.gemm_last_config()
+    assert splits == 1 and csplit > 1, (plan, splits, csplit)
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K)
+    assert check(values_f64(C), Cref, R, out_bf16=False)["ok"]
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch(capi):
     # 4099 x 4099 packed A and B need ~67 MB of padded copies: more than the 32 MiB scratch.
     n = 4099
