@@ -62,7 +62,37 @@ struct DevInfo {
     int major = 0;
     int minor = 0;
     unsigned int* status = nullptr;  // device address of g_pw_status
+    // Clusters of 2, 4 and 8 CTAs (one CTA per SM: the GEMM kernels' shared memory) that the
+    // device holds at once; a cluster must sit inside one GPC, so this is below sms / size.
+    int cluster_cap[3] = {0, 0, 0};
 };
+
+// Empty kernel with the GEMM kernels' footprint (one CTA per SM), for the cluster occupancy query.
+__global__ void cluster_probe_kernel() {}
+constexpr int kProbeSmemBytes = 200 * 1024;
+
+// Clusters of `cdim` CTAs of one SM each that the device can hold at once (sms / cdim if the
+// query fails).
+int query_cluster_cap(int sms, int cdim) {
+    static bool attr = cudaFuncSetAttribute(cluster_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            kProbeSmemBytes) == cudaSuccess;
+    int n = 0;
+    if (attr) {
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3((unsigned)cdim, 1, 1);
+        q.blockDim = dim3(192, 1, 1);
+        q.dynamicSmemBytes = kProbeSmemBytes;
+        cudaLaunchAttribute qa[1];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = (unsigned)cdim;
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        q.attrs = qa;
+        q.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, cluster_probe_kernel, &q) != cudaSuccess) n = 0;
+    }
+    return n > 0 && n <= sms / cdim ? n : sms / cdim;
+}
 
 std::mutex g_dev_mu;
 std::array<DevInfo, kMaxDevices> g_dev;
@@ -81,6 +111,7 @@ bool device_info(int dev, DevInfo& out) {
         if (d.major == 10 && d.minor == 0) {
             if (cudaGetSymbolAddress(&st, g_pw_status) != cudaSuccess || st == nullptr) return false;
             d.status = static_cast<unsigned int*>(st);
+            for (int i = 0; i < 3; ++i) d.cluster_cap[i] = query_cluster_cap(d.sms, 2 << i);
         }
         d.init = true;
     }
@@ -328,27 +359,31 @@ CUtensorMapDataType out_dtype(int out) {
 constexpr int kMaxSplits = 8;
 constexpr int kMinSplitKBlocks = 8;
 // Operand bytes one CTA pulls through TMA per second when its tiles are not compute-bound
-// (measured on B200 with few, deep tiles: 8192x256x4096, 1024x1024x8192).
-constexpr double kCtaOperandBytesPerSec = 140e9;
+// (fitted on B200 to few, deep tiles: 8192x256x4096, 127x8191x2048, 512^2 x 8192, 1024^2 x 8192,
+// 2048^2 x 8192, every streaming plan, unsplit and cut across a cluster).
+constexpr double kCtaOperandBytesPerSec = 100e9;
+// Time of a tile that its mainloop does not cover: the first loads' latency and the epilogue
+// (the same fit).  A persistent launch pays it once (later tiles overlap their epilogue with
+// the next mainloop); cluster split-K, whose CTAs hold one tile each, once per wave.
+constexpr double kTileFixedSec = 10e-6;
 // Split-K cost per unit, measured on B200: a fixed part (counter, fences, the longer fixup
 // epilogue), the write of the unit's fp32 partial sums and the last unit's read of the others.
 constexpr double kSplitFixedSec = 4e-6;
 constexpr double kSplitWriteBytesPerSec = 45e9;
 constexpr double kSplitReadBytesPerSec = 90e9;
-// Fixed cost of one launch that the waves do not cover: pipeline fill, the exposed epilogue of
-// the last tiles and teardown.  Fitted on B200 to single-wave shapes (2048^3, 8192x512x4096,
-// 8192x256x4096, 127x8191x2048), where 2-CTA tiles pay more (the leader waits for both CTAs'
-// loads) and plan 1 beats plan 2 by 13 % although their waves model equal.
-constexpr double kLaunchFixedSecOneCta = 3e-6;
-constexpr double kLaunchFixedSecCtaPair = 6e-6;
+// Fixed cost of one launch besides kTileFixedSec: launch latency, prologue and teardown.
+// 2-CTA tiles pay more (the leader waits for both CTAs' loads; on B200 plan 1 beats plan 2 by
+// 13 % on 2048^3 although their waves model equal).
+constexpr double kLaunchFixedSecOneCta = 5e-6;
+constexpr double kLaunchFixedSecCtaPair = 8e-6;
 // Split-K arrival counters per CTA and tile: one per epilogue warp.
 constexpr int kSplitCountersPerCta = 4;
 // Cluster split-K: a tile's K slices run on the CTAs of one cluster (2, 4 or 8 CTAs) and their
-// partial tiles are added through distributed shared memory.  Cost per tile beyond its slice's
-// mainloop: two cluster barriers and the partial-tile write (fixed), and each CTA's read of the
-// other slices' share of its part of the tile.
-constexpr double kClusterSplitFixedSec = 4e-6;
-constexpr double kClusterSplitBytesPerSec = 150e9;
+// partial tiles are added through distributed shared memory.  Cost per wave beyond its slices'
+// mainloop and kTileFixedSec: each CTA's read of the other slices' share of its part of the
+// tile, at the per-warp rate distributed shared memory gives the reduction (fitted with the
+// constants above).
+constexpr double kClusterSplitBytesPerSec = 25e9;
 
 // Can plan `i` serve this request?
 bool plan_serves(int i, const Req& r) {
@@ -378,7 +413,7 @@ double plan_time(int i, const Req& r, int sms, int splits) {
     const double compute = 2.0 * (double)(tm * tn) * unit_k / (pd.rate * 1e12 / (double)slots);
     const double stream = (double)(tm + tn) * unit_k * 2.0 / (pd.cg * kCtaOperandBytesPerSec);
     double t = (double)cdiv(plan_tiles(pd, r) * splits, slots) * (compute > stream ? compute : stream) +
-               (pd.cg == 2 ? kLaunchFixedSecCtaPair : kLaunchFixedSecOneCta);
+               (pd.cg == 2 ? kLaunchFixedSecCtaPair : kLaunchFixedSecOneCta) + kTileFixedSec;
     if (splits > 1) {
         const double partial = 128.0 * (double)tn * 4.0;  // bytes per CTA and unit
         t += kSplitFixedSec + partial / kSplitWriteBytesPerSec + (splits - 1) * partial / kSplitReadBytesPerSec;
@@ -406,25 +441,27 @@ int forced_splits() {
     return 0;
 }
 
-// Plans whose kernels take cluster split-K: one-CTA streaming tiles with one MMA sub-tile
-// (the kernel's Tile::CSPLIT_OK).
-bool plan_csplit_ok(const PlanDesc& pd) { return pd.cg == 1 && pd.nsub == 1 && !pd.ares; }
+// Plans whose kernels take cluster split-K: streaming tiles with one MMA sub-tile (the kernel's
+// Tile::CSPLIT_OK), sliced over up to 8 CTAs per cluster (CTA pairs: up to 4 slices).
+bool plan_csplit_ok(const PlanDesc& pd) { return pd.nsub == 1 && !pd.ares; }
+int max_csplit(const PlanDesc& pd) { return 8 / pd.cg; }
 
-// Modelled time (s) of plan `i` with cluster split-K over `cs` CTAs: the tiles' clusters run in
-// waves of sms / cs clusters, each CTA streaming its K slice; then the reduction.
-double plan_time_csplit(int i, const Req& r, int sms, int cs) {
+// Modelled time (s) of plan `i` with cluster split-K over `cs` slices (CTAs or CTA pairs): the
+// tiles' clusters run in waves of `cap` clusters (as many as the device holds at once), each
+// slice streaming its K range; then the tile's fixed cost and the reduction.
+double plan_time_csplit(int i, const Req& r, int sms, int cs, int cap) {
     const PlanDesc& pd = kPlans[i];
     const long long tm = 128LL * pd.cg, tn = (long long)pd.bn * pd.nsub;
     const long long kb = cdiv(cdiv(r.K, pd.bk), cs);
     const double unit_k = (double)(kb * pd.bk);
-    const long long slots = sms;  // one CTA per SM
+    const long long slots = sms / pd.cg;  // one CTA per SM
     const double compute = 2.0 * (double)(tm * tn) * unit_k / (pd.rate * 1e12 / (double)slots);
-    const double stream = (double)(tm + tn) * unit_k * 2.0 / kCtaOperandBytesPerSec;
-    const long long waves = cdiv(plan_tiles(pd, r), sms / cs);
+    const double stream = (double)(tm + tn) * unit_k * 2.0 / (pd.cg * kCtaOperandBytesPerSec);
+    const long long waves = cdiv(plan_tiles(pd, r), cap > 0 ? cap : 1);
     const double xbytes = 128.0 * (double)tn * 4.0 * (double)(cs - 1) / (double)cs;
-    return (double)waves * ((compute > stream ? compute : stream) + kClusterSplitFixedSec +
+    return (double)waves * ((compute > stream ? compute : stream) + kTileFixedSec +
                             xbytes / kClusterSplitBytesPerSec) +
-           kLaunchFixedSecOneCta;
+           (pd.cg == 2 ? kLaunchFixedSecCtaPair : kLaunchFixedSecOneCta);
 }
 
 // GEMM_BF16_CLUSTER_SPLIT=s (2, 4 or 8) forces cluster split-K with s slices wherever the plan
@@ -438,9 +475,10 @@ int forced_csplit() {
     return 0;
 }
 
-// Plan and K split for a request on a device with `sms` SMs (auto unless overridden); without
-// `allow_split` no global split-K (it needs workspace); cluster split-K needs none.
-Choice choose(const Req& r, int sms, bool allow_split) {
+// Plan and K split for a request on a device with `sms` SMs that holds `ccap[i]` clusters of
+// 2 << i CTAs at once (auto unless overridden); without `allow_split` no global split-K (it
+// needs workspace); cluster split-K needs none.
+Choice choose(const Req& r, int sms, const int* ccap, bool allow_split) {
     const int fs_env = forced_splits();  // GEMM_BF16_SPLIT_K (0: unset)
     const int fs = allow_split ? fs_env : 1;
     const int fcs = r.index != nullptr ? 1 : forced_csplit();  // dedup units replace K slices
@@ -477,14 +515,17 @@ Choice choose(const Req& r, int sms, bool allow_split) {
             if (!plan_csplit_ok(pd)) continue;
             if (only >= 0 ? i != only : (pd.rate <= 0.0 || !plan_serves(i, r))) continue;
             const long long tiles = plan_tiles(pd, r);
-            for (int cs = 2; cs <= 8; cs *= 2) {
+            for (int cs = 2; cs <= max_csplit(pd); cs *= 2) {
                 if (fcs > 0 && cs != fcs) continue;
                 if (!split_valid(pd, r, cs) || cdiv(r.K, pd.bk) < (long long)cs * 2) continue;
+                const int cdim = cs * pd.cg;
+                const int cap = ccap[cdim == 2 ? 0 : cdim == 4 ? 1 : 2];
                 // Automatically only where the unsplit tiles leave at least half the SMs idle and
-                // the split tiles still fit in one wave: measured on B200, a split that adds a
-                // wave (8192x256x4096: 37.8 -> 50 us) or only fills the last SMs loses.
-                if (fcs == 0 && (2 * tiles > sms || tiles * cs > sms)) continue;
-                const double t = plan_time_csplit(i, r, sms, cs);
+                // the split tiles' clusters all fit on the device at once: measured on B200, a
+                // split that adds a wave (8192x256x4096: 37.8 -> 50 us) or only fills the last
+                // SMs loses.
+                if (fcs == 0 && (2 * tiles * pd.cg > sms || tiles > cap)) continue;
+                const double t = plan_time_csplit(i, r, sms, cs, cap);
                 if (fcs > 0 || (t < cbar && t < best_t * 0.999)) {
                     best = {i, 1, cs};
                     best_t = t;
@@ -704,12 +745,13 @@ gemm_status_t run(Req r, Workspace wsrc) {
         ch = *r.force;
         if (ch.plan < 0 || ch.plan >= kNumPlans || !plan_serves(ch.plan, rg)) return GEMM_ERR_INVALID_ARG;
         if (ch.splits > 1 && (!may_split || !split_valid(kPlans[ch.plan], rg, ch.splits))) return GEMM_ERR_INVALID_ARG;
-        if (ch.csplit > 1 && (dedup || !plan_csplit_ok(kPlans[ch.plan]) || !split_valid(kPlans[ch.plan], rg, ch.csplit)))
+        if (ch.csplit > 1 && (dedup || !plan_csplit_ok(kPlans[ch.plan]) || ch.csplit > max_csplit(kPlans[ch.plan]) ||
+                              !split_valid(kPlans[ch.plan], rg, ch.csplit)))
             return GEMM_ERR_INVALID_ARG;
     } else if (!overrides_set() && tuned_choice(key, &tuned) && (tuned.splits <= 1 || may_split)) {
         ch = tuned;
     } else {
-        ch = choose(rg, di.sms, may_split);
+        ch = choose(rg, di.sms, di.cluster_cap, may_split);
     }
     // Split-K partial sums (fp32, one 128 x tile_n slab per CTA, tile and slice) and the
     // per-(tile, CTA, epilogue warp) arrival counters, which must start at zero.
@@ -889,7 +931,7 @@ std::vector<Choice> candidates(const Req& rg, int sms, bool dedup) {
         for (int s = 2; s <= kMaxSplits; s *= 2) {
             if (!split_valid(pd, rg, s) || cdiv(rg.K, pd.bk) < (long long)s * 2) continue;
             c.push_back(Choice{i, s, 1, kGroupM});
-            if (plan_csplit_ok(pd)) c.push_back(Choice{i, 1, s, kGroupM});
+            if (plan_csplit_ok(pd) && s <= max_csplit(pd)) c.push_back(Choice{i, 1, s, kGroupM});
         }
     }
     return c;
@@ -1109,7 +1151,8 @@ gemm_status_t gemm_tuning_load(const char* path) {
              (k.b_mn | k.in_f16 | k.c_read | k.a_ok | k.b_ok | k.c_tma) <= 1 && k.out >= OUT_F32 &&
              k.out <= OUT_F16 && v.ch.splits >= 1 && v.ch.splits <= kMaxSplits &&
              (v.ch.csplit == 1 || v.ch.csplit == 2 || v.ch.csplit == 4 || v.ch.csplit == 8) &&
-             !(v.ch.splits > 1 && v.ch.csplit > 1) && (v.ch.csplit == 1 || plan_csplit_ok(*pd)) &&
+             !(v.ch.splits > 1 && v.ch.csplit > 1) &&
+             (v.ch.csplit == 1 || (plan_csplit_ok(*pd) && v.ch.csplit <= max_csplit(*pd))) &&
              (v.ch.splits == 1 || !pd->ares) && v.ch.group_m >= 1 && v.ch.group_m <= 64;
         if (ok) rows.emplace_back(k, v);
     }

@@ -168,9 +168,9 @@ struct Tile {
     static_assert(BK == 64 || BK == 32, "stage K");
     static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
     // Cluster split-K: after its K slice, a CTA's ring is idle and holds its 128 x BN fp32
-    // partial tile for the other CTAs of the cluster to read.
+    // partial tile (its rows of the tile, every column) for the other slices' CTAs to read.
     static constexpr int XCHG_BYTES = 128 * BN * 4;
-    static constexpr bool CSPLIT_OK = CG == 1 && NSUB == 1 && ARES == 0 && XCHG_BYTES <= STAGES * STAGE_BYTES;
+    static constexpr bool CSPLIT_OK = NSUB == 1 && ARES == 0 && XCHG_BYTES <= STAGES * STAGE_BYTES;
     static_assert(ARES == 0 || BK == 64, "resident A uses K=64 blocks");
 };
 
@@ -189,18 +189,19 @@ __device__ __forceinline__ void decode_tile(const KParams& p, int t, int& b, int
     nb = w / gm;
 }
 
+// `ctarank` is the CTA's rank in its cluster; with CG == 2 its pair partner is ctarank ^ 1.
 template <int CG>
-__device__ __forceinline__ void raise_abort(uint32_t slot_abort, uint32_t rank, unsigned int* status,
+__device__ __forceinline__ void raise_abort(uint32_t slot_abort, uint32_t ctarank, unsigned int* status,
                                             unsigned int code) {
     atomicOr(status, code);
     st_shared_volatile_u32(slot_abort, 1u);
-    if constexpr (CG == 2) st_cluster_u32(map_to_rank(slot_abort, rank ^ 1u), 1u);
+    if constexpr (CG == 2) st_cluster_u32(map_to_rank(slot_abort, ctarank ^ 1u), 1u);
 }
 
 // Slow path of wait_phase: poll with the global-timer bound.
 template <int CG, bool CLUSTER_SCOPE>
 __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, uint32_t slot_abort,
-                                             uint32_t rank, unsigned int* status,
+                                             uint32_t ctarank, unsigned int* status,
                                              unsigned long long timeout_ns, unsigned int code) {
     const uint64_t t0 = global_timer_ns();
     for (;;) {
@@ -210,7 +211,7 @@ __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, uint
                 return true;
         if (ld_shared_volatile_u32(slot_abort) != 0u) return false;
         if (global_timer_ns() - t0 > timeout_ns) {
-            raise_abort<CG>(slot_abort, rank, status, code);
+            raise_abort<CG>(slot_abort, ctarank, status, code);
             return false;
         }
     }
@@ -221,10 +222,10 @@ __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, uint
 // critical path (a stage that is already full or free) it costs one instruction.
 template <int CG, bool CLUSTER_SCOPE>
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, uint32_t slot_abort,
-                                           uint32_t rank, unsigned int* status,
+                                           uint32_t ctarank, unsigned int* status,
                                            unsigned long long timeout_ns, unsigned int code) {
     if (CLUSTER_SCOPE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    return wait_phase_slow<CG, CLUSTER_SCOPE>(bar, parity, slot_abort, rank, status, timeout_ns, code);
+    return wait_phase_slow<CG, CLUSTER_SCOPE>(bar, parity, slot_abort, ctarank, status, timeout_ns, code);
 }
 
 template <int CG, int BN, int NSUB, int STAGES, int BK, int B_MN, int OUT, int ARES>
@@ -239,13 +240,16 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
 
     const uint32_t warp = threadIdx.x >> 5;
     const uint32_t lane = threadIdx.x & 31u;
-    const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
-    // Cluster split-K: the grid holds one cluster of CS CTAs per tile; CTA crank of the cluster
-    // computes K slice crank of the tile.  Otherwise a persistent grid of CG-CTA clusters.
+    // Cluster split-K: the grid holds one cluster of CS K slices per tile, each slice a CTA (CG ==
+    // 1) or a CTA pair (CG == 2; pairs are cluster ranks 2j, 2j+1), slice crank computing k-blocks
+    // [crank*kb_per_split, ...).  Otherwise a persistent grid of CG-CTA clusters.
     const int CS = (T::CSPLIT_OK && p.csplit > 1) ? p.csplit : 1;
-    const uint32_t crank = CS > 1 ? cluster_ctarank() : 0u;
-    const int cluster_id = CS > 1 ? (int)(blockIdx.x / CS) : (int)(blockIdx.x / CG);
-    const int num_clusters = CS > 1 ? (int)(gridDim.x / CS) : (int)(gridDim.x / CG);
+    const uint32_t ctarank = (CG == 2 || CS > 1) ? cluster_ctarank() : 0u;
+    const uint32_t rank = CG == 2 ? (ctarank & 1u) : 0u;     // rank in the CTA pair
+    const uint32_t pair0 = CG == 2 ? (ctarank & ~1u) : 0u;   // cluster rank of the pair's leader
+    const uint32_t crank = CS > 1 ? ctarank / CG : 0u;       // K slice (cluster split-K)
+    const int cluster_id = (int)(blockIdx.x / (CG * CS));
+    const int num_clusters = (int)(gridDim.x / (CG * CS));
     // K blocks of work unit u (global split-K: unit = (tile, slice); cluster split-K: this CTA's
     // slice of the tile; else all of K).
     const int SG = (ARES == 0 && p.splits > 1) ? p.splits : 1;
@@ -297,7 +301,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint32_t full_leader0 = CG == 2 ? map_to_rank(bar_full(0), 0) : bar_full(0);
+            const uint32_t full_leader0 = CG == 2 ? map_to_rank(bar_full(0), pair0) : bar_full(0);
             // A and B panels are read by several CTAs of a wave: keep them in L2 (build options
             // PW_OPERAND_L2_POLICY for A and PW_B_L2_POLICY for B: 0 evict-normal, 1 evict-last,
             // 2 evict-first).
@@ -312,7 +316,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             if (ARES != 0 && ok) {
                 // This CTA's 128 rows of the single M tile, every k-block, once.
                 if (rank == 0) mbar_arrive_expect_tx(bar_ares, (uint32_t)(T::A_BYTES * CG * p.k_blocks));
-                const uint32_t ares_bar = CG == 2 ? map_to_rank(bar_ares, 0) : bar_ares;
+                const uint32_t ares_bar = CG == 2 ? map_to_rank(bar_ares, pair0) : bar_ares;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     const uint32_t sa = sbase + T::OFF_A + kb * T::A_BYTES;
                     if constexpr (CG == 1) tma_load_3d(sa, &tmA, ares_bar, kb * T::BK, (int)rank * 128, 0, pol);
@@ -328,7 +332,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 decode_tile(p, t, b, mb, nb);
                 const int a_row = mb * T::BM + (int)rank * 128;
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
-                    if (!wait_phase<CG, false>(bar_empty(stage), phase ^ 1u, slot_abort, rank,
+                    if (!wait_phase<CG, false>(bar_empty(stage), phase ^ 1u, slot_abort, ctarank,
                                                p.status, p.timeout_ns, kStatusProducer)) {
                         ok = false;
                         break;
@@ -377,17 +381,17 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             const uint64_t adesc0 = smem_desc(sbase + T::OFF_A, 16, T::KMAJ_SBO, T::KMAJ_SWIZZLE);
             const uint64_t bdesc0 = B_MN ? smem_desc(sbase + T::OFF_B, T::MN_BOX_BYTES, 1024, 2u)
                                          : smem_desc(sbase + T::OFF_B, 16, T::KMAJ_SBO, T::KMAJ_SWIZZLE);
-            const uint32_t empty_r0 = CG == 2 ? map_to_rank(bar_empty(0), 0) : bar_empty(0);
-            const uint32_t empty_r1 = CG == 2 ? map_to_rank(bar_empty(0), 1) : bar_empty(0);
-            const uint32_t tfull_r0 = CG == 2 ? map_to_rank(bar_tfull(0), 0) : bar_tfull(0);
-            const uint32_t tfull_r1 = CG == 2 ? map_to_rank(bar_tfull(0), 1) : bar_tfull(0);
+            const uint32_t empty_r0 = CG == 2 ? map_to_rank(bar_empty(0), pair0) : bar_empty(0);
+            const uint32_t empty_r1 = CG == 2 ? map_to_rank(bar_empty(0), pair0 + 1u) : bar_empty(0);
+            const uint32_t tfull_r0 = CG == 2 ? map_to_rank(bar_tfull(0), pair0) : bar_tfull(0);
+            const uint32_t tfull_r1 = CG == 2 ? map_to_rank(bar_tfull(0), pair0 + 1u) : bar_tfull(0);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t tph = 0u;  // bit i: phase of accumulator slot i's next use
             int acc = 0;                 // slot of the tile when NSUB == 1
             bool ok = true;
             if constexpr (ARES != 0) {
-                ok = wait_phase<CG, false>(bar_ares, 0u, slot_abort, rank, p.status, p.timeout_ns, kStatusMma);
+                ok = wait_phase<CG, false>(bar_ares, 0u, slot_abort, ctarank, p.status, p.timeout_ns, kStatusMma);
                 tc_fence_after();
             }
             const int S = UPT;
@@ -412,7 +416,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 int kb_lo, kb_hi;
                 unit_k(u, kb_lo, kb_hi);
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
-                    if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, rank, p.status, p.timeout_ns,
+                    if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, ctarank, p.status, p.timeout_ns,
                                                kStatusMma)) {
                         ok = false;
                         break;
@@ -426,7 +430,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                         const int slot = NSUB == 1 ? acc : sub;
                         if (kb == kb_lo) {
                             // the slot must have been drained by the epilogue of its last use
-                            if (!wait_phase<CG, CG == 2>(bar_tempty(slot), ((tph >> slot) & 1u) ^ 1u, slot_abort, rank,
+                            if (!wait_phase<CG, CG == 2>(bar_tempty(slot), ((tph >> slot) & 1u) ^ 1u, slot_abort, ctarank,
                                                          p.status, p.timeout_ns, kStatusMma)) {
                                 ok = false;
                                 break;
@@ -466,7 +470,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         const int half = ew / 4;                      // which part of the slot's columns
         constexpr int CPW = T::CHUNKS / T::EPI_HALVES;  // chunks per warp and slot
         const uint32_t stg = sbase + T::OFF_STG + ew * T::STG_BUFS * T::STG_BYTES;
-        const uint32_t tempty_leader0 = CG == 2 ? map_to_rank(bar_tempty(0), 0) : bar_tempty(0);
+        const uint32_t tempty_leader0 = CG == 2 ? map_to_rank(bar_tempty(0), pair0) : bar_tempty(0);
         uint32_t tph = 0u;
         int acc = 0;
         int buf = 0;
@@ -739,9 +743,11 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             __syncwarp();
         };
         const int S = SG;  // global split-K: streaming plans only
-        // Cluster split-K exchange buffer: the ring, as 4 KiB pieces (32 rows x 32 fp32 columns,
-        // the staging-buffer image), piece (32-column block cb, lane quarter qq) at
-        // ((cb * 4 + qq) << 12).
+        // Cluster split-K exchange buffer: the ring, as 4 KiB pieces (32 rows x 32 fp32 columns),
+        // piece (32-column block cb, lane quarter qq) at ((cb * 4 + qq) << 12).  Inside a piece,
+        // columns 4j..4j+3 of row r sit at j * 512 + r * 16: a warp-wide 16-byte access then
+        // covers 512 contiguous bytes, the form distributed shared memory serves fastest
+        // (measured on B200: about 3x the rate of the same loads 128 bytes apart).
         const uint32_t xchg = sbase + T::OFF_A;
         for (int u = cluster_id; ok && u < p.tiles * UPT; u += num_clusters) {
             const int t = u / UPT;
@@ -782,7 +788,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 const int slot = NSUB == 1 ? acc : sub;
                 int w_ok = 1;
                 if (lane == 0)
-                    w_ok = wait_phase<CG, false>(bar_tfull(slot), (tph >> slot) & 1u, slot_abort, rank, p.status, p.timeout_ns,
+                    w_ok = wait_phase<CG, false>(bar_tfull(slot), (tph >> slot) & 1u, slot_abort, ctarank, p.status, p.timeout_ns,
                                                  kStatusEpilogue);
                 w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
                 if (!w_ok) {
@@ -802,10 +808,10 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                         if (ci == 0) fence_proxy_async_smem();
 #pragma unroll
                         for (int h = 0; h < PIECES; ++h) {
-                            const uint32_t pc = xchg + ((uint32_t)((c * PIECES + h) * 4 + q) << 12) + lane * 128u;
+                            const uint32_t pc = xchg + ((uint32_t)((c * PIECES + h) * 4 + q) << 12) + lane * 16u;
 #pragma unroll
                             for (int j = 0; j < 8; ++j)
-                                st_shared_v4(pc + ((uint32_t)(j ^ (int)(lane & 7u)) << 4), __float_as_uint(v[32 * h + 4 * j]),
+                                st_shared_v4(pc + (uint32_t)j * 512u, __float_as_uint(v[32 * h + 4 * j]),
                                              __float_as_uint(v[32 * h + 4 * j + 1]), __float_as_uint(v[32 * h + 4 * j + 2]),
                                              __float_as_uint(v[32 * h + 4 * j + 3]));
                         }
@@ -945,10 +951,11 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         if constexpr (T::CSPLIT_OK) {
             if (CS > 1) {
                 // Cluster split-K reduction.  Once every CTA of the cluster has its partial tile in
-                // its shared memory, the cluster's 4*CS epilogue warps share the tile's (lane quarter,
-                // column chunk) items; each adds the CS partials of its item in slice order
-                // 0..CS-1, reading them through distributed shared memory, and runs the normal
-                // alpha/beta epilogue on the sum.  The result does not depend on timing.
+                // its shared memory, the 4*CS epilogue warps of the CTAs holding the same 128 rows
+                // (one per slice) share those rows' (lane quarter, column chunk) items; each adds
+                // the CS partials of its item in slice order 0..CS-1, reading them through
+                // distributed shared memory, and runs the normal alpha/beta epilogue on the sum.
+                // The result does not depend on timing.
                 __syncwarp();
                 cluster_sync();
                 if (ok && ld_shared_volatile_u32(slot_abort) == 0u) {
@@ -957,18 +964,18 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     constexpr int CH = BN / T::STG_COLS;  // column chunks of the tile
                     for (int it = (int)crank * 4 + ew; it < 4 * CH; it += 4 * CS) {
                         const int qq = it & 3, c = it >> 2;
-                        const int row0 = mb * T::BM + 32 * qq;
+                        const int row0 = mb * T::BM + (int)rank * 128 + 32 * qq;
                         float v[T::STG_COLS];
 #pragma unroll 1
                         for (int s2 = 0; s2 < CS; ++s2) {
-                            const uint32_t src = map_to_rank(xchg, (uint32_t)s2) + lane * 128u;
+                            // slice s2's CTA holding the same rows of the tile
+                            const uint32_t src = map_to_rank(xchg, (uint32_t)(s2 * CG) + rank) + lane * 16u;
 #pragma unroll
                             for (int h = 0; h < PIECES; ++h) {
                                 uint32_t x[8][4];
 #pragma unroll
                                 for (int j = 0; j < 8; ++j)
-                                    ld_cluster_v4(src + ((uint32_t)((c * PIECES + h) * 4 + qq) << 12) +
-                                                      ((uint32_t)(j ^ (int)(lane & 7u)) << 4),
+                                    ld_cluster_v4(src + ((uint32_t)((c * PIECES + h) * 4 + qq) << 12) + (uint32_t)j * 512u,
                                                   x[j][0], x[j][1], x[j][2], x[j][3]);
 #pragma unroll
                                 for (int j = 0; j < 8; ++j)

@@ -61,12 +61,12 @@ gemm_status_t launch_persistent(const LaunchArgs& a) {
         max_clusters[dev].store(clusters);
         attr_done[dev].store(1);
     }
-    // Cluster split-K: one cluster of csplit CTAs per tile (not persistent: each CTA computes
-    // one K slice of one tile).  Otherwise a persistent grid of CG-CTA clusters, at most as many
-    // as fit on the device at once.
+    // Cluster split-K: one cluster of csplit slices per tile, a slice being a CTA or a CTA pair
+    // (not persistent: each CTA computes one K slice of one tile).  Otherwise a persistent grid of
+    // CG-CTA clusters, at most as many as fit on the device at once.
     const bool csplit = T::CSPLIT_OK && a.p.csplit > 1;
     if (a.p.csplit > 1 && !csplit) return GEMM_ERR_UNSUPPORTED;
-    const int cdim = csplit ? a.p.csplit : CG;
+    const int cdim = csplit ? a.p.csplit * CG : CG;
     long long ctas;
     if (csplit) {
         ctas = (long long)a.p.tiles * cdim;

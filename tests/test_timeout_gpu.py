@@ -31,7 +31,8 @@ def capi():
 # (plan, forced split): the persistent plans, and K cut across a cluster (every CTA of the cluster
 # must still reach both cluster barriers) or through the workspace.
 CASES = [(0, None), (2, None), (4, None), (5, None), (1, ("GEMM_BF16_CLUSTER_SPLIT", "2")),
-         (0, ("GEMM_BF16_CLUSTER_SPLIT", "4")), (0, ("GEMM_BF16_SPLIT_K", "2"))]
+         (0, ("GEMM_BF16_CLUSTER_SPLIT", "4")), (2, ("GEMM_BF16_CLUSTER_SPLIT", "2")),
+         (3, ("GEMM_BF16_CLUSTER_SPLIT", "4")), (0, ("GEMM_BF16_SPLIT_K", "2"))]
 
 
 @pytest.mark.parametrize("case", CASES, ids=[f"plan{p}" + (f"_{e[0][10:]}{e[1]}" if e else "") for p, e in CASES])
