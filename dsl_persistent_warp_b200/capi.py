@@ -168,7 +168,8 @@ def gemm_tuning_load(path: str) -> int:
 
 
 def gemm_last_config() -> tuple[int, int, int, int]:
-    """(plan, workspace K slices, cluster K slices, raster group) of this thread's last launch."""
+    """(plan, workspace K slices (0: stream-K), cluster K slices, raster group) of this thread's
+    last launch."""
     v = [ctypes.c_int(0) for _ in range(4)]
     st = LIB.gemm_last_config(*[ctypes.byref(x) for x in v])
     if st != GEMM_OK:

@@ -155,6 +155,7 @@ struct Choice {
     int splits;       // global split-K slices (1: none)
     int csplit = 1;   // cluster split-K slices (1: none)
     int group_m = 0;  // m-blocks per raster group (0: the default)
+    int sk = 0;       // 1: stream-K (the last, partial wave's tiles cut into K ranges over every cluster)
 };
 
 // One request, in the batched form (batch == 1 for the plain GEMM).
@@ -441,6 +442,46 @@ int forced_splits() {
     return 0;
 }
 
+// GEMM_BF16_STREAM_K=1 forces stream-K wherever it applies (tests, tuning); 0 forbids it; unset
+// leaves the choice to the model.
+int forced_stream_k() {
+    const char* e = std::getenv("GEMM_BF16_STREAM_K");
+    if (e && (e[0] == '0' || e[0] == '1') && e[1] == '\0') return e[0] == '1' ? 1 : 2;
+    return 0;  // 0: unset, 1: forced, 2: forbidden
+}
+
+// Stream-K geometry of a plan for a request: the persistent grid's clusters, the tiles of the
+// last, partial wave (computed as K ranges spread evenly over every cluster; the whole tiles
+// come after them in the tile order) and the most ranges one of those tiles is cut into (its
+// partial-sum slots).  sk_tiles == 0: stream-K does not apply (at most one wave, whole waves
+// only, or ranges shorter than kMinSplitKBlocks k-blocks).
+struct SkGeom {
+    int clusters = 0;
+    int sk_tiles = 0;
+    int max_parts = 0;
+};
+SkGeom sk_geometry(const PlanDesc& pd, const Req& r, int clusters) {
+    SkGeom g;
+    const long long tiles = plan_tiles(pd, r), kb = cdiv(r.K, pd.bk);
+    if (pd.ares || clusters <= 0 || tiles <= clusters) return g;
+    const long long sk = tiles % clusters;
+    const long long total = sk * kb;
+    if (sk == 0 || total < (long long)clusters * kMinSplitKBlocks) return g;
+    const long long base = total / clusters, extra = total % clusters, edge = extra * (base + 1);
+    auto owner = [&](long long i) { return i < edge ? i / (base + 1) : extra + (i - edge) / base; };
+    long long mp = 1;
+    for (long long t = 0; t < sk; ++t) {
+        const long long n = owner((t + 1) * kb - 1) - owner(t * kb) + 1;
+        if (n > mp) mp = n;
+    }
+    g.clusters = clusters;
+    g.sk_tiles = (int)sk;
+    g.max_parts = (int)mp;
+    return g;
+}
+// Persistent clusters of a plan on the device (one CTA per SM; CTA pairs as the device places them).
+int persistent_clusters(const PlanDesc& pd, int sms, const int* ccap) { return pd.cg == 2 ? ccap[0] : sms; }
+
 // Plans whose kernels take cluster split-K: streaming tiles with one MMA sub-tile (the kernel's
 // Tile::CSPLIT_OK), sliced over up to 8 CTAs per cluster (CTA pairs: up to 4 slices).
 bool plan_csplit_ok(const PlanDesc& pd) { return pd.nsub == 1 && !pd.ares; }
@@ -473,6 +514,28 @@ int forced_csplit() {
         if (v == 1 || v == 2 || v == 4 || v == 8) return v;
     }
     return 0;
+}
+
+// Modelled time (s) of plan `i` with stream-K geometry `g`: the whole waves and the last wave's
+// share of K per cluster, the fixed costs of a launch, and the exposed part of the fixup (the
+// last part of a tile reads every part's partial sums; the publishing overlaps the next unit).
+double plan_time_sk(int i, const Req& r, int sms, const SkGeom& g) {
+    const PlanDesc& pd = kPlans[i];
+    const long long tm = 128LL * pd.cg, tn = (long long)pd.bn * pd.nsub;
+    const double unit_k = (double)(cdiv(r.K, pd.bk) * pd.bk);
+    const long long slots = sms / pd.cg;
+    const double compute = 2.0 * (double)(tm * tn) * unit_k / (pd.rate * 1e12 / (double)slots);
+    const double stream = (double)(tm + tn) * unit_k * 2.0 / (pd.cg * kCtaOperandBytesPerSec);
+    const long long tiles = plan_tiles(pd, r);
+    const double waves = (double)((tiles - g.sk_tiles) / g.clusters) + (double)g.sk_tiles / (double)g.clusters;
+    const double partial = 128.0 * (double)tn * 4.0;
+    // A tile of two MMA sub-tiles holds both accumulator slots, so the next unit's mainloop
+    // waits while a part's partial sums are published (measured on B200: 4096^3 and
+    // 2048x8192x8192 on plan 4 gained nothing from stream-K).
+    const double units = (double)g.sk_tiles * (double)g.max_parts / (double)g.clusters;
+    const double publish = pd.nsub == 2 ? units * partial / kSplitWriteBytesPerSec : 0.0;
+    return waves * (compute > stream ? compute : stream) + (pd.cg == 2 ? kLaunchFixedSecCtaPair : kLaunchFixedSecOneCta) +
+           kTileFixedSec + kSplitFixedSec + (double)g.max_parts * partial / kSplitReadBytesPerSec + publish;
 }
 
 // Plan and K split for a request on a device with `sms` SMs that holds `ccap[i]` clusters of
@@ -535,6 +598,25 @@ Choice choose(const Req& r, int sms, const int* ccap, bool allow_split) {
         }
     }
     if (fs > 0 || !allow_split || best.csplit > 1) return best;
+    // Stream-K where the last wave is partial: forced, or where it beats the best by 5 %.
+    const int fsk = r.index != nullptr ? 2 : forced_stream_k();
+    if (fsk != 2) {
+        const double sk_bar = best_t * 0.95;
+        Choice sk_best{-1, 1};
+        double sk_t = 0.0;
+        for (int i = 0; i < kNumPlans; ++i) {
+            const PlanDesc& pd = kPlans[i];
+            if (only >= 0 ? i != only : (pd.rate <= 0.0 || !plan_serves(i, r))) continue;
+            const SkGeom g = sk_geometry(pd, r, persistent_clusters(pd, sms, ccap));
+            if (g.sk_tiles == 0) continue;
+            const double t = plan_time_sk(i, r, sms, g);
+            if (sk_best.plan < 0 || t < sk_t) sk_best = Choice{i, 1, 1, 0, 1}, sk_t = t;
+        }
+        // forced: the plan chosen so far, where stream-K applies to it
+        if (fsk == 1 && sk_geometry(kPlans[best.plan], r, persistent_clusters(kPlans[best.plan], sms, ccap)).sk_tiles > 0)
+            return Choice{best.plan, 1, 1, 0, 1};
+        if (sk_best.plan >= 0 && (fsk == 1 || sk_t < sk_bar)) return sk_best;
+    }
     const double split_bar = best_t * 0.90;
     for (int i = 0; i < kNumPlans; ++i) {
         const PlanDesc& pd = kPlans[i];
@@ -748,7 +830,11 @@ gemm_status_t run(Req r, Workspace wsrc) {
         if (ch.csplit > 1 && (dedup || !plan_csplit_ok(kPlans[ch.plan]) || ch.csplit > max_csplit(kPlans[ch.plan]) ||
                               !split_valid(kPlans[ch.plan], rg, ch.csplit)))
             return GEMM_ERR_INVALID_ARG;
-    } else if (!overrides_set() && tuned_choice(key, &tuned) && (tuned.splits <= 1 || may_split)) {
+        if (ch.sk && (!may_split || ch.splits > 1 || ch.csplit > 1 ||
+                      sk_geometry(kPlans[ch.plan], rg, persistent_clusters(kPlans[ch.plan], di.sms, di.cluster_cap))
+                              .sk_tiles == 0))
+            return GEMM_ERR_INVALID_ARG;
+    } else if (!overrides_set() && tuned_choice(key, &tuned) && ((tuned.splits <= 1 && !tuned.sk) || may_split)) {
         ch = tuned;
     } else {
         ch = choose(rg, di.sms, di.cluster_cap, may_split);
@@ -759,9 +845,16 @@ gemm_status_t run(Req r, Workspace wsrc) {
     const PlanDesc pd = kPlans[plan];
     const long long tiles_est = plan_tiles(pd, rg);
     size_t ws_p = 0, ws_n = 0;
-    if (ch.splits > 1) {
-        ws_p = (size_t)tiles_est * pd.cg * ch.splits * 128 * pd.bn * pd.nsub * sizeof(float);
-        ws_n = (size_t)round_up(tiles_est * pd.cg * kSplitCountersPerCta * (long long)sizeof(unsigned int), 256);
+    SkGeom skg;
+    if (ch.sk) skg = sk_geometry(pd, rg, persistent_clusters(pd, di.sms, di.cluster_cap));
+    if (ch.sk && skg.sk_tiles == 0) return GEMM_ERR_INVALID_ARG;  // a tuned entry that no longer applies
+    const bool partials = ch.splits > 1 || ch.sk;
+    if (partials) {
+        // slots for split-K's slices of every tile, or stream-K's parts of the cut tiles
+        const long long ptiles = ch.sk ? skg.sk_tiles : tiles_est;
+        const int parts = ch.sk ? skg.max_parts : ch.splits;
+        ws_p = (size_t)ptiles * pd.cg * parts * 128 * pd.bn * pd.nsub * sizeof(float);
+        ws_n = (size_t)round_up(ptiles * pd.cg * kSplitCountersPerCta * (long long)sizeof(unsigned int), 256);
     }
     // Deduplicated form: per-entry item lists (offsets, cursor scratch, items).
     size_t ws_d = 0;
@@ -786,9 +879,9 @@ gemm_status_t run(Req r, Workspace wsrc) {
         if (pooled) cudaFreeAsync(ws, r.stream);
         return s;
     };
-    float* ws_partials = ch.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + ws_a + ws_b) : nullptr;
+    float* ws_partials = partials ? reinterpret_cast<float*>(static_cast<char*>(ws) + ws_a + ws_b) : nullptr;
     unsigned int* ws_counters =
-        ch.splits > 1 ? reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + ws_a + ws_b + ws_p) : nullptr;
+        partials ? reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + ws_a + ws_b + ws_p) : nullptr;
     if (ws_n && cudaMemsetAsync(ws_counters, 0, ws_n, r.stream) != cudaSuccess) return fail(GEMM_ERR_CUDA);
     int* dd_off = nullptr;
     int* dd_dst = nullptr;
@@ -867,6 +960,13 @@ gemm_status_t run(Req r, Workspace wsrc) {
         p.splits = ch.splits;
         p.kb_per_split = (int)cdiv(p.k_blocks, ch.splits);
         p.ws = ws_partials;
+        p.ws_parts = ch.splits;
+        p.counters = ws_counters;
+    } else if (ch.sk) {
+        p.sk_tiles = skg.sk_tiles;
+        p.sk_clusters = skg.clusters;
+        p.ws = ws_partials;
+        p.ws_parts = skg.max_parts;
         p.counters = ws_counters;
     } else if (ch.csplit > 1) {
         p.csplit = ch.csplit;
@@ -901,7 +1001,8 @@ gemm_status_t run(Req r, Workspace wsrc) {
     p.timeout_ns = g_timeout_ns.load();
     p.test_stall = test_stall_requested() ? 1 : 0;
     st = launch_by_plan(plan, la);
-    if (st == GEMM_OK) t_last = Choice{plan, p.splits > 1 ? p.splits : 1, p.csplit > 1 ? p.csplit : 1, p.group_m};
+    if (st == GEMM_OK)
+        t_last = Choice{plan, p.splits > 1 ? p.splits : 1, p.csplit > 1 ? p.csplit : 1, p.group_m, p.sk_tiles > 0 ? 1 : 0};
     if (pooled) cudaFreeAsync(ws, r.stream);
     return st;
 }
@@ -918,7 +1019,7 @@ gemm_status_t guarded(const Req& r, Workspace w) {
 // are), unsplit and with each valid split of K through the workspace (2, 4, 8 slices) or across
 // a cluster (2, 4, 8 CTAs, one-CTA plans), and raster groups of 8, 16 and 32 m-blocks when the
 // tiles fill more than two waves.
-std::vector<Choice> candidates(const Req& rg, int sms, bool dedup) {
+std::vector<Choice> candidates(const Req& rg, int sms, const int* ccap, bool dedup) {
     std::vector<Choice> c;
     for (int i = 0; i < kNumPlans; ++i) {
         const PlanDesc& pd = kPlans[i];
@@ -927,6 +1028,8 @@ std::vector<Choice> candidates(const Req& rg, int sms, bool dedup) {
         const bool many_waves = tiles > 2LL * (sms / pd.cg);
         const int groups[3] = {16, 8, 32};
         for (int g = 0; g < (many_waves ? 3 : 1); ++g) c.push_back(Choice{i, 1, 1, groups[g]});
+        if (!dedup && sk_geometry(pd, rg, persistent_clusters(pd, sms, ccap)).sk_tiles > 0)
+            c.push_back(Choice{i, 1, 1, kGroupM, 1});
         if (pd.ares || dedup || many_waves) continue;
         for (int s = 2; s <= kMaxSplits; s *= 2) {
             if (!split_valid(pd, rg, s) || cdiv(rg.K, pd.bk) < (long long)s * 2) continue;
@@ -953,7 +1056,7 @@ gemm_status_t autotune(Req r, float* best_us) {
     const TuneKey key = tune_key(r, di.sms);
     Req rg = r;
     if (dedup) rg.batch = r.n_x;
-    const std::vector<Choice> cand = candidates(rg, di.sms, dedup);
+    const std::vector<Choice> cand = candidates(rg, di.sms, di.cluster_cap, dedup);
     if (cand.empty()) return GEMM_ERR_UNSUPPORTED;
 
     // Scratch C: the whole extent of the caller's C, at the same offset from a 256-byte
@@ -1117,7 +1220,7 @@ gemm_status_t gemm_tuning_save(const char* path) {
             const TuneVal& v = kv.second;
             std::fprintf(f, "gemmtune1 %d %d %d %d %d %d %d %d %d %d %d %d %d %d %d %d %d %.3f\n", k.sms, k.batch, k.M,
                          k.N, k.K, k.n_x, k.b_mn, k.in_f16, k.out, k.c_read, k.a_ok, k.b_ok, k.c_tma, v.ch.plan,
-                         v.ch.splits, v.ch.csplit, v.ch.group_m, (double)v.us);
+                         v.ch.sk ? 0 : v.ch.splits, v.ch.csplit, v.ch.group_m, (double)v.us);
         }
     }
     return std::fclose(f) == 0 ? GEMM_OK : GEMM_ERR_INVALID_ARG;
@@ -1145,6 +1248,10 @@ gemm_status_t gemm_tuning_load(const char* path) {
                                   &k.b_ok, &k.c_tma, &v.ch.plan, &v.ch.splits, &v.ch.csplit, &v.ch.group_m, &us,
                                   &consumed);
         v.us = (float)us;
+        if (n == 18 && v.ch.splits == 0) {  // stream-K
+            v.ch.splits = 1;
+            v.ch.sk = 1;
+        }
         const PlanDesc* pd = (v.ch.plan >= 0 && v.ch.plan < kNumPlans) ? &kPlans[v.ch.plan] : nullptr;
         ok = n == 18 && line[consumed] == '\0' && pd != nullptr && k.sms > 0 && k.batch >= 1 && k.M >= 1 &&
              k.N >= 1 && k.K >= 1 && k.n_x >= 0 && (k.b_mn | k.in_f16 | k.c_read | k.a_ok | k.b_ok | k.c_tma) >= 0 &&
@@ -1153,7 +1260,8 @@ gemm_status_t gemm_tuning_load(const char* path) {
              (v.ch.csplit == 1 || v.ch.csplit == 2 || v.ch.csplit == 4 || v.ch.csplit == 8) &&
              !(v.ch.splits > 1 && v.ch.csplit > 1) &&
              (v.ch.csplit == 1 || (plan_csplit_ok(*pd) && v.ch.csplit <= max_csplit(*pd))) &&
-             (v.ch.splits == 1 || !pd->ares) && v.ch.group_m >= 1 && v.ch.group_m <= 64;
+             (v.ch.splits == 1 || !pd->ares) && !(v.ch.sk && (pd->ares || v.ch.csplit > 1)) && v.ch.group_m >= 1 &&
+             v.ch.group_m <= 64;
         if (ok) rows.emplace_back(k, v);
     }
     std::fclose(f);
@@ -1166,7 +1274,7 @@ gemm_status_t gemm_tuning_load(const char* path) {
 gemm_status_t gemm_last_config(int* plan, int* splits, int* csplit, int* group_m) {
     if (!plan || !splits || !csplit || !group_m) return GEMM_ERR_INVALID_ARG;
     *plan = t_last.plan;
-    *splits = t_last.splits;
+    *splits = t_last.sk ? 0 : t_last.splits;
     *csplit = t_last.csplit;
     *group_m = t_last.group_m;
     return GEMM_OK;

@@ -93,8 +93,13 @@ struct KParams {
     int csplit;              // cluster split-K (one-CTA plans): K slices per tile, computed by the
                              // csplit CTAs of one thread-block cluster, one slice each; the partial
                              // sums are added through distributed shared memory (<= 1: none)
-    float* ws;               // split-K partials: per (tile, CTA rank, slice) the CTA's 128 rows x
+    int sk_tiles;            // stream-K: tiles [0, sk_tiles) are computed as K ranges spread evenly
+                             // over sk_clusters clusters (0: none), the rest whole
+    int sk_clusters;         // stream-K: clusters of the grid (the launch has exactly this many)
+    float* ws;               // split-K partials: per (tile, CTA rank, part) the CTA's 128 rows x
                              // TILE_N columns in fp32, as 4 KiB pieces per epilogue warp
+    int ws_parts;            // partial slots per (tile, CTA rank): splits, or stream-K's most
+                             // K ranges of one tile
     unsigned int* counters;  // split-K arrivals per (tile, CTA rank, epilogue warp); zero on entry,
                              // and the last arrival puts it back to zero
     // Deduplicated batches (shared-W form): the tiles cover the batch_real distinct X entries;
@@ -256,10 +261,54 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
     // Work units per tile: global split-K slices, or the deduplicated form's destination parts.
     const int DS = (p.dd_off != nullptr && p.dsplit > 1) ? p.dsplit : 1;
     const int UPT = SG > 1 ? SG : DS;
-    auto unit_k = [&](int u, int& kb_lo, int& kb_hi) {
-        const int sl = SG > 1 ? u % SG : (int)crank;
-        kb_lo = (SG > 1 || CS > 1) ? sl * p.kb_per_split : 0;
+    // Stream-K: the k-blocks of tiles [0, sk_tiles) form one sequence of sk_tiles * k_blocks
+    // iterations, cut into sk_clusters contiguous ranges of equal length (the first `extra` one
+    // longer); a tile crossed by several ranges is computed in parts, one per range, and added up
+    // by the split-K fixup.  Each cluster runs its range's parts first, then whole tiles
+    // sk_tiles + cluster_id, + num_clusters, ...  (This is the persistent tile walk with its last,
+    // partial wave spread over every cluster.)
+    const int SK = (ARES == 0 && CS == 1 && SG == 1 && DS == 1 && p.sk_tiles > 0) ? 1 : 0;
+    const long long sk_total = (long long)p.sk_tiles * p.k_blocks;
+    const long long sk_base = SK ? sk_total / p.sk_clusters : 0;
+    const long long sk_extra = SK ? sk_total % p.sk_clusters : 0;
+    auto sk_start = [&](long long c) { return c * sk_base + (c < sk_extra ? c : sk_extra); };
+    auto sk_owner = [&](long long i) {  // the range holding iteration i
+        const long long edge = sk_extra * (sk_base + 1);
+        return i < edge ? i / (sk_base + 1) : sk_extra + (i - edge) / (sk_base > 0 ? sk_base : 1);
+    };
+    const long long sk_lo = SK ? sk_start(cluster_id) : 0, sk_hi = SK ? sk_start(cluster_id + 1) : 0;
+    const int sk_t0 = (int)(sk_lo / (SK ? p.k_blocks : 1));
+    const int sk_units = (SK && sk_hi > sk_lo) ? (int)((sk_hi - 1) / p.k_blocks) - sk_t0 + 1 : 0;
+    // Work unit i of this cluster: tile t, k-blocks [kb_lo, kb_hi), part `part` of `parts` whose
+    // partial sums the split-K fixup adds (parts == 1: the whole tile; deduplicated batches: part
+    // is the destination part and parts 1).  False past the last unit.
+    auto get_unit = [&](int i, int& t, int& kb_lo, int& kb_hi, int& part, int& parts) -> bool {
+        if (SK) {
+            if (i < sk_units) {
+                t = sk_t0 + i;
+                const long long ts = (long long)t * p.k_blocks, te = ts + p.k_blocks;
+                kb_lo = (int)((sk_lo > ts ? sk_lo : ts) - ts);
+                kb_hi = (int)((sk_hi < te ? sk_hi : te) - ts);
+                const long long first = sk_owner(ts);
+                part = (int)(cluster_id - first);
+                parts = (int)(sk_owner(te - 1) - first) + 1;
+                return true;
+            }
+            t = p.sk_tiles + cluster_id + (i - sk_units) * num_clusters;
+            kb_lo = 0;
+            kb_hi = p.k_blocks;
+            part = 0;
+            parts = 1;
+            return t < p.tiles;
+        }
+        const int u = cluster_id + i * num_clusters;
+        t = u / UPT;
+        const int sl = u % UPT;
+        kb_lo = (SG > 1 || CS > 1) ? (SG > 1 ? sl : (int)crank) * p.kb_per_split : 0;
         kb_hi = (SG > 1 || CS > 1) ? min(p.k_blocks, kb_lo + p.kb_per_split) : p.k_blocks;
+        part = sl;
+        parts = SG;
+        return u < p.tiles * UPT;
     };
 
     const uint32_t bar0 = sbase + T::OFF_BAR;
@@ -323,11 +372,8 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     else tma_load_3d_pair(sa, &tmA, ares_bar, kb * T::BK, (int)rank * 128, 0, pol);
                 }
             }
-            const int S = UPT;
-            for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters) {
-                const int t = u / S;
-                int kb_lo, kb_hi;
-                unit_k(u, kb_lo, kb_hi);
+            int t, kb_lo, kb_hi, part, parts;
+            for (int i = 0; ok && get_unit(i, t, kb_lo, kb_hi, part, parts); ++i) {
                 int b, mb, nb;
                 decode_tile(p, t, b, mb, nb);
                 const int a_row = mb * T::BM + (int)rank * 128;
@@ -394,7 +440,6 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 ok = wait_phase<CG, false>(bar_ares, 0u, slot_abort, ctarank, p.status, p.timeout_ns, kStatusMma);
                 tc_fence_after();
             }
-            const int S = UPT;
             auto commit_tfull = [&](int slot) {
                 // accumulator of this slot complete: hand it to the epilogue
                 if constexpr (CG == 1) {
@@ -412,9 +457,8 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     umma_commit<2>(empty_r1 + 8u * st);
                 }
             };
-            for (int u = cluster_id; ok && u < p.tiles * S; u += num_clusters) {
-                int kb_lo, kb_hi;
-                unit_k(u, kb_lo, kb_hi);
+            int t, kb_lo, kb_hi, part, parts;
+            for (int i = 0; ok && get_unit(i, t, kb_lo, kb_hi, part, parts); ++i) {
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!wait_phase<CG, false>(bar_full(stage), phase, slot_abort, ctarank, p.status, p.timeout_ns,
                                                kStatusMma)) {
@@ -742,16 +786,16 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             }
             __syncwarp();
         };
-        const int S = SG;  // global split-K: streaming plans only
         // Cluster split-K exchange buffer: the ring, as 4 KiB pieces (32 rows x 32 fp32 columns),
         // piece (32-column block cb, lane quarter qq) at ((cb * 4 + qq) << 12).  Inside a piece,
         // columns 4j..4j+3 of row r sit at j * 512 + r * 16: a warp-wide 16-byte access then
         // covers 512 contiguous bytes, the form distributed shared memory serves fastest
         // (measured on B200: about 3x the rate of the same loads 128 bytes apart).
         const uint32_t xchg = sbase + T::OFF_A;
-        for (int u = cluster_id; ok && u < p.tiles * UPT; u += num_clusters) {
-            const int t = u / UPT;
-            const int sl = u % UPT;  // split-K slice, or destination part of a deduplicated batch
+        // per unit: tile t, part sl of S (split-K slice or stream-K range; or the destination part
+        // of a deduplicated batch, S == 1)
+        int t, kb_lo_u, kb_hi_u, sl, S;
+        for (int i = 0; ok && get_unit(i, t, kb_lo_u, kb_hi_u, sl, S); ++i) {
             int b, mb, nb;
             decode_tile(p, t, b, mb, nb);
             const int row0 = mb * T::BM + (int)rank * 128 + 32 * q;
@@ -778,7 +822,9 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     }
             }
             // this warp's partials of slice s of the tile: pieces in (sub, ci, piece) order
-            auto slab = [&](int s) { return p.ws + ((size_t)(t * CG + (int)rank) * S + s) * WS_TILE + (size_t)ew * WS_WARP; };
+            auto slab = [&](int s) {
+                return p.ws + ((size_t)(t * CG + (int)rank) * p.ws_parts + s) * WS_TILE + (size_t)ew * WS_WARP;
+            };
             if (S > 1) {
                 // the staging buffer must not be read by a tensor store still in flight
                 if (lane == 0) bulk_wait_group_read<0>();
@@ -858,7 +904,13 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                             }
                         }
                     } else {
-                        // publish this slice's partial sums; the slot stays held for the fixup
+                        // publish this part's partial sums; the slot is free once its last chunk
+                        // is read, so the next unit's mainloop overlaps the publishing and fixup
+                        if (ci == CPW - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * slot);
+                        }
                         float* g = slab(sl) + (size_t)((sub * CPW + ci) * PIECES) * 1024;
 #pragma unroll
                         for (int h = 0; h < PIECES; ++h) put_piece(g + h * 1024, v + 32 * h, stg + buf * T::STG_BYTES);
@@ -867,9 +919,9 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
             }
             if (S > 1 && ok) {
                 // Split-K fixup, per warp (its 32 rows).  Arrival is counted after the partial
-                // sums are visible; the last of the S slices to arrive adds them up in slice
-                // order 0..S-1, its own from TMEM, the others from global memory, so the result
-                // is the same whatever the arrival order.  Nothing waits on another CTA.
+                // sums are visible; the last of the S parts to arrive adds them up in part order
+                // 0..S-1, reading every one (its own too) from global memory, so the result is the
+                // same whatever the arrival order.  Nothing waits on another CTA.
                 __threadfence();
                 __syncwarp();
                 unsigned int* cnt = p.counters + ((size_t)(t * CG + (int)rank) * T::EPI_WARPS + ew);
@@ -882,8 +934,6 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                 if (old == (unsigned int)(S - 1)) {
                     __threadfence();
                     for (int sub = 0; sub < NSUB; ++sub) {
-                        const int slot = NSUB == 1 ? acc : sub;
-                        const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(slot * BN);
 #pragma unroll 1
                         for (int ci = 0; ci < CPW; ++ci) {
                             const int c = half * CPW + ci;
@@ -897,13 +947,6 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                             const uint32_t sb = stg + buf * T::STG_BYTES;
 #pragma unroll 1
                             for (int s2 = 0; s2 < S; ++s2) {
-                                if (s2 == sl) {
-                                    float own[T::STG_COLS];
-                                    load_chunk(trow, c, own);
-#pragma unroll
-                                    for (int j = 0; j < T::STG_COLS; ++j) v[j] += own[j];
-                                    continue;
-                                }
                                 // every piece of the chunk in flight at once, then through the buffer
                                 const uint4* g = reinterpret_cast<const uint4*>(slab(s2) + off);
                                 uint4 x[PIECES][8];
@@ -934,16 +977,6 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                             finish_chunk(b, nb, row0, row, sub, c, v);
                         }
                     }
-                }
-            }
-            if (S > 1) {
-                // the unit's accumulator slots are free again
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    if (NSUB == 1) mbar_arrive_cluster(tempty_leader0 + 8u * acc);
-                    else
-                        for (int sub = 0; sub < NSUB; ++sub) mbar_arrive_cluster(tempty_leader0 + 8u * sub);
                 }
             }
             if (NSUB == 1) acc ^= 1;

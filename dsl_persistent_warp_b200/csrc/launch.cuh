@@ -70,6 +70,11 @@ gemm_status_t launch_persistent(const LaunchArgs& a) {
     long long ctas;
     if (csplit) {
         ctas = (long long)a.p.tiles * cdim;
+    } else if (a.p.sk_tiles > 0) {
+        // stream-K: exactly the clusters its K ranges were cut for (correct even if fewer fit at
+        // once: no CTA waits for another)
+        if (a.p.sk_clusters <= 0) return GEMM_ERR_INVALID_ARG;
+        ctas = (long long)a.p.sk_clusters * CG;
     } else {
         const int upt = a.p.splits > 1 ? a.p.splits : (a.p.dd_off != nullptr && a.p.dsplit > 1) ? a.p.dsplit : 1;
         const long long units = (long long)a.p.tiles * upt;  // work units

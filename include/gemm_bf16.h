@@ -180,18 +180,23 @@ GEMM_API gemm_status_t gemm_bf16_device_status(struct CUstream_st* stream);
  * call is replaced by the automatic choice for that call.
  *
  * With few output tiles and a long K, the kernels may also cut K into slices, in one of two ways:
- *   cluster split-K (plans 0, 1 and 8): the 2, 4 or 8 slices of a tile run on the CTAs of one
- *     thread-block cluster, which add their partial tiles through distributed shared memory
- *     (no workspace, so gemm_bf16_noalloc may use it too);
+ *   cluster split-K (plans 0-3 and 8): the 2, 4 or 8 slices of a tile run on the CTAs of one
+ *     thread-block cluster (plans 2 and 3: 2 or 4 slices, each on a CTA pair), which add their
+ *     partial tiles through distributed shared memory (no workspace, so gemm_bf16_noalloc may
+ *     use it too);
  *   split-K through the workspace (plans 0-4 and 8): each (tile, slice) unit writes fp32
  *     partial sums to the workspace and the last unit of a tile adds them.
- * Both add the slices in slice order, so results stay bitwise reproducible.  The plan and the
- * slice count come from a cost model; environment variables read at every call override it for
+ * With more tiles than the device runs at once and a partial last wave, stream-K (plans 0-4 and
+ * 8; workspace) spreads the last wave's tiles over every cluster as equal ranges of k-blocks;
+ * a tile cut by several ranges is added up like a workspace split.
+ * All of them add the parts in a fixed order, so results stay bitwise reproducible.  The plan and
+ * the split come from a cost model; environment variables read at every call override it for
  * sweeps and tests:
  *   GEMM_BF16_SPLIT_K=s        (1..8) s workspace slices wherever the plan and K allow it
  *                              (1: no split of either kind unless the next variable forces one)
  *   GEMM_BF16_CLUSTER_SPLIT=s  (2, 4, 8) cluster split-K with s slices where the plan takes it;
  *                              1: never cluster split-K
+ *   GEMM_BF16_STREAM_K=1       stream-K wherever it applies; 0: never
  *   GEMM_BF16_GROUP_M=g        (1..64) m-blocks per group of the persistent tile order
  */
 GEMM_API gemm_status_t gemm_bf16_set_plan(int plan);
@@ -291,7 +296,8 @@ GEMM_API int gemm_tuning_size(void);
  * entries to it (same key: replaced).  One line per problem:
  *   gemmtune1 sms batch M N K n_unique b_mn in_f16 out c_read a_ok b_ok c_tma plan splits csplit group_m us
  * (b_mn: batched forms; c_read: beta != 0; a_ok/b_ok: operand read in place by TMA; c_tma: C
- * stored by TMA; splits: workspace K slices; csplit: cluster K slices; us: measured time).
+ * stored by TMA; splits: workspace K slices, 0 for stream-K; csplit: cluster K slices; us:
+ * measured time).
  * Lines starting with '#' and empty lines are skipped.  A file that cannot be opened, or any
  * malformed line or impossible configuration, returns GEMM_ERR_INVALID_ARG and loads nothing.
  */
@@ -300,7 +306,8 @@ GEMM_API gemm_status_t gemm_tuning_load(const char* path);
 
 /*
  * gemm_last_config -- the configuration of the calling thread's most recent GEMM kernel launch
- * (plan, workspace K slices, cluster K slices, raster group); plan -1 before any launch.
+ * (plan, workspace K slices -- 0 for stream-K --, cluster K slices, raster group); plan -1 before
+ * any launch.
  * GEMM_ERR_INVALID_ARG if a pointer is NULL.
  */
 GEMM_API gemm_status_t gemm_last_config(int* plan, int* splits, int* csplit, int* group_m);

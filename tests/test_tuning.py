@@ -10,6 +10,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 GOOD = """# tuned on a B200 (148 SMs)
 gemmtune1 148 1 1024 1024 8192 0 0 0 1 1 1 1 1 1 1 4 8 31.250
 gemmtune1 148 2048 256 128 512 0 1 0 1 0 1 1 1 7 1 1 8 80.500
+gemmtune1 148 1 4096 4096 4096 0 0 0 1 0 1 1 1 4 0 1 16 95.000
 """
 
 
@@ -32,13 +33,13 @@ def test_tuning_table_round_trip(capi, tmp_path):
     src = tmp_path / "in.txt"
     src.write_text(GOOD)
     assert capi.gemm_tuning_load(str(src)) == capi.GEMM_OK
-    assert capi.gemm_tuning_size() == 2
+    assert capi.gemm_tuning_size() == 3
     out = tmp_path / "out.txt"
     assert capi.gemm_tuning_save(str(out)) == capi.GEMM_OK
     assert _lines(out) == _lines(src)
     # loading the same file again replaces, it does not duplicate
     assert capi.gemm_tuning_load(str(out)) == capi.GEMM_OK
-    assert capi.gemm_tuning_size() == 2
+    assert capi.gemm_tuning_size() == 3
     assert capi.gemm_tuning_clear() == capi.GEMM_OK
     assert capi.gemm_tuning_size() == 0
 
@@ -48,6 +49,8 @@ BAD_LINES = [
     "gemmtune1 148 1 1024 1024 8192 0 0 0 1 1 1 1 1 4 1 2 8 1.0",     # plan 4 takes no cluster split
     "gemmtune1 148 1 1024 1024 8192 0 0 0 1 1 1 1 1 1 2 2 8 1.0",     # two kinds of split at once
     "gemmtune1 148 1 1024 1024 8192 0 0 0 1 1 1 1 1 7 2 1 8 1.0",     # resident-A plan with a split
+    "gemmtune1 148 1 1024 1024 8192 0 0 0 1 1 1 1 1 7 0 1 8 1.0",     # resident-A plan with stream-K
+    "gemmtune1 148 1 1024 1024 8192 0 0 0 1 1 1 1 1 1 0 2 8 1.0",     # stream-K and a cluster split
     "gemmtune1 148 1 1024 1024 8192 0 0 0 3 1 1 1 1 1 1 1 8 1.0",     # unknown output type
     "gemmtune1 148 1 1024 1024 8192 0 0 0 1 1 1 1 1 1 1 3 8 1.0",     # cluster split of 3
     "gemmtune1 148 1 1024 1024 8192 0 0 0 1 1 1 1 1 1 1 1 8",         # missing time
