@@ -378,7 +378,7 @@ constexpr double kSplitReadBytesPerSec = 90e9;
 constexpr double kLaunchFixedSecOneCta = 5e-6;
 constexpr double kLaunchFixedSecCtaPair = 8e-6;
 // Split-K arrival counters per CTA and tile: one per epilogue warp.
-constexpr int kSplitCountersPerCta = 4;
+constexpr int kSplitCountersPerCta = 8;
 // Cluster split-K: a tile's K slices run on the CTAs of one cluster (2, 4 or 8 CTAs) and their
 // partial tiles are added through distributed shared memory.  Cost per wave beyond its slices'
 // mainloop and kTileFixedSec: each CTA's read of the other slices' share of its part of the
