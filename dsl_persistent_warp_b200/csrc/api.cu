@@ -176,6 +176,7 @@ struct Req {
     // index[b] (device memory, `batch` ints); nullptr for the plain forms.
     const int* index = nullptr;
     int n_x = 0;
+    int items = 0;  // planning copies of a deduplicated request: the output items (batch = n_x)
     // A configuration to run as is (the autotuner's candidates); nullptr: choose one.
     const Choice* force = nullptr;
 };
@@ -452,9 +453,10 @@ int forced_stream_k() {
 
 // Stream-K geometry of a plan for a request: the persistent grid's clusters, the tiles of the
 // last, partial wave (computed as K ranges spread evenly over every cluster; the whole tiles
-// come after them in the tile order) and the most ranges one of those tiles is cut into (its
-// partial-sum slots).  sk_tiles == 0: stream-K does not apply (at most one wave, whole waves
-// only, or ranges shorter than kMinSplitKBlocks k-blocks).
+// come after them in the tile order) and a bound on the ranges one of those tiles is cut into
+// (its partial-sum slots): a tile's kb consecutive k-blocks meet at most ceil((kb-1)/base) + 1
+// ranges of at least `base` k-blocks each.  sk_tiles == 0: stream-K does not apply (at most one
+// wave, whole waves only, or ranges shorter than kMinSplitKBlocks k-blocks).
 struct SkGeom {
     int clusters = 0;
     int sk_tiles = 0;
@@ -467,13 +469,9 @@ SkGeom sk_geometry(const PlanDesc& pd, const Req& r, int clusters) {
     const long long sk = tiles % clusters;
     const long long total = sk * kb;
     if (sk == 0 || total < (long long)clusters * kMinSplitKBlocks) return g;
-    const long long base = total / clusters, extra = total % clusters, edge = extra * (base + 1);
-    auto owner = [&](long long i) { return i < edge ? i / (base + 1) : extra + (i - edge) / base; };
-    long long mp = 1;
-    for (long long t = 0; t < sk; ++t) {
-        const long long n = owner((t + 1) * kb - 1) - owner(t * kb) + 1;
-        if (n > mp) mp = n;
-    }
+    const long long base = total / clusters;
+    long long mp = cdiv(kb - 1, base) + 1;
+    if (mp > clusters) mp = clusters;
     g.clusters = clusters;
     g.sk_tiles = (int)sk;
     g.max_parts = (int)mp;
@@ -550,6 +548,12 @@ Choice choose(const Req& r, int sms, const int* ccap, bool allow_split) {
     if (forced >= 0 && plan_serves(forced, r)) {
         if (kPlans[forced].ares) return {forced, 1};
         only = forced;
+    } else if (r.index != nullptr && r.b_mn && r.K <= 1024 && r.items >= 32LL * r.n_x && plan_serves(8, r)) {
+        // Deduplicated batches with few distinct entries (32 or more items each) are bound by
+        // writing the items: the smallest one-CTA tiles spread the writes over the most SMs
+        // (B200, 2048 items of 256x128 from 256x512 . 512x128: 16 entries 47.4 -> 43.4 us with
+        // plan 8 instead of plan 7, 64 entries 47.4 -> 45.3 us; at 256 entries plan 7 wins).
+        return {8, 1};
     } else if (r.b_mn && r.K <= 1024 && pack_factor(kPlans[2], r.b_mn, r.N) > 1) {
         // Shared-W batched shapes with short K are bound by streaming X and Y through HBM: a
         // 256x256 tile holding several batch entries side by side, with W resident in shared
@@ -704,7 +708,30 @@ TuneKey tune_key(const Req& r, int sms) {
 // the table off for the call.
 bool overrides_set() {
     return g_plan_override.load() >= 0 || std::getenv("GEMM_BF16_SPLIT_K") != nullptr ||
-           std::getenv("GEMM_BF16_CLUSTER_SPLIT") != nullptr || std::getenv("GEMM_BF16_GROUP_M") != nullptr;
+           std::getenv("GEMM_BF16_CLUSTER_SPLIT") != nullptr || std::getenv("GEMM_BF16_GROUP_M") != nullptr ||
+           std::getenv("GEMM_BF16_STREAM_K") != nullptr;
+}
+
+// The cost model's choice per problem (and workspace permission), so that a repeated call skips
+// the model.  Not used while an override is set; bounded by clearing it when it grows large.
+std::mutex g_memo_mu;
+std::unordered_map<TuneKey, Choice, TuneKeyHash> g_memo[2];
+constexpr size_t kMemoMax = 4096;
+
+bool memo_choice(const TuneKey& k, bool may_split, Choice* out) {
+    std::lock_guard<std::mutex> lk(g_memo_mu);
+    auto& m = g_memo[may_split ? 1 : 0];
+    auto it = m.find(k);
+    if (it == m.end()) return false;
+    *out = it->second;
+    return true;
+}
+
+void memo_store(const TuneKey& k, bool may_split, const Choice& c) {
+    std::lock_guard<std::mutex> lk(g_memo_mu);
+    auto& m = g_memo[may_split ? 1 : 0];
+    if (m.size() >= kMemoMax) m.clear();
+    m[k] = c;
 }
 
 // ------------------------------------------------------------------ auxiliary launches
@@ -798,7 +825,7 @@ gemm_status_t run(Req r, Workspace wsrc) {
     // stores each entry's result to the r.batch output items that use it.
     const bool dedup = r.index != nullptr;
     Req rg = r;
-    if (dedup) rg.batch = r.n_x;
+    if (dedup) rg.batch = r.n_x, rg.items = r.batch;
 
     // Operands TMA cannot read as given go through a padded, 16-byte aligned copy; C that TMA
     // cannot address takes the row-by-row store path.
@@ -836,8 +863,11 @@ gemm_status_t run(Req r, Workspace wsrc) {
             return GEMM_ERR_INVALID_ARG;
     } else if (!overrides_set() && tuned_choice(key, &tuned) && ((tuned.splits <= 1 && !tuned.sk) || may_split)) {
         ch = tuned;
-    } else {
+    } else if (overrides_set()) {
         ch = choose(rg, di.sms, di.cluster_cap, may_split);
+    } else if (!memo_choice(key, may_split, &ch)) {
+        ch = choose(rg, di.sms, di.cluster_cap, may_split);
+        memo_store(key, may_split, ch);
     }
     // Split-K partial sums (fp32, one 128 x tile_n slab per CTA, tile and slice) and the
     // per-(tile, CTA, epilogue warp) arrival counters, which must start at zero.
@@ -1055,7 +1085,7 @@ gemm_status_t autotune(Req r, float* best_us) {
     normalize(r);
     const TuneKey key = tune_key(r, di.sms);
     Req rg = r;
-    if (dedup) rg.batch = r.n_x;
+    if (dedup) rg.batch = r.n_x, rg.items = r.batch;
     const std::vector<Choice> cand = candidates(rg, di.sms, di.cluster_cap, dedup);
     if (cand.empty()) return GEMM_ERR_UNSUPPORTED;
 

@@ -11,8 +11,8 @@ import pytest
 import torch
 
 import oracle
-from parity import bits_of, check, sample_rows, to_dev_bf16, values_f64
-from synth import bf16_bits_to_f64, f64_to_bf16_bits, matrix_bf16
+from parity import bits_of, check, sample_rows, to_dev_bf16, to_dev_f16, values_f64
+from synth import bf16_bits_to_f64, f64_to_bf16_bits, matrix_bf16, matrix_f16
 
 pytestmark = pytest.mark.gpu
 
@@ -97,4 +97,44 @@ def test_stream_k_is_refused_where_it_does_not_apply(pw):
     assert cfg[1] != 0
     Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, rows=sample_rows(M, seed=5))
     rep = check(values_f64(C[torch.as_tensor(sample_rows(M, seed=5), device="cuda")]), Cref, R, out_bf16=False)
+    assert rep["ok"], rep
+
+
+@pytest.mark.parametrize("plan", [4, 2])
+def test_stream_k_batched_shared_w(pw, plan):
+    """Stream-K on the batched shared-W call (MN-major X), alpha/beta with Y in place."""
+    batch, M, K = 8, 1000, 2048
+    N = 2048 if plan == 4 else 1024  # 128 tiles either way: more than the 74 CTA pairs
+    assert pw.capi.gemm_bf16_set_plan(plan) == 0
+    W = matrix_bf16(1600 + plan, M, K, std=K ** -0.5)
+    X = matrix_bf16(1610 + plan, batch * K, N)
+    y0 = torch.randn(batch, M, N, dtype=torch.float32, generator=torch.Generator().manual_seed(plan))
+    y0 = y0.to(torch.bfloat16)
+    Y = y0.clone().cuda()
+    pw.gemm_bf16_batched_shared_w(to_dev_bf16(W), to_dev_bf16(X).view(batch, K, N), Y, alpha=0.5, beta=1.0)
+    torch.cuda.synchronize()
+    assert pw.device_status() == 0
+    _require_stream_k(pw.capi.gemm_last_config()[:3], plan)
+    rows = sample_rows(M, seed=plan)
+    Cref, R = oracle.gemm_batched(W, X, batch=batch, M=M, N=N, K=K, stride_x=K * N,
+                                  y0=y0.to(torch.float32).numpy().reshape(batch * M, N), stride_y=M * N,
+                                  alpha=0.5, beta=1.0, rows=rows)
+    got = values_f64(Y[:, torch.as_tensor(rows, device="cuda")])
+    rep = check(got, Cref, R, out_bf16=True)
+    assert rep["ok"], rep
+
+
+def test_stream_k_fp16_operands_fp32_out(pw):
+    """fp16 operands and fp32 output (the two-sub-tile plan's chunk-by-chunk epilogue)."""
+    M, N, K = CASES[4]
+    assert pw.capi.gemm_bf16_set_plan(4) == 0
+    A, B = matrix_f16(1700, M, K), matrix_f16(1701, N, K)
+    C = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    pw.gemm_bf16(to_dev_f16(A), to_dev_f16(B), C)
+    torch.cuda.synchronize()
+    assert pw.device_status() == 0
+    _require_stream_k(pw.capi.gemm_last_config()[:3], 4)
+    rows = sample_rows(M, seed=17)
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, rows=rows, in_dtype="f16")
+    rep = check(values_f64(C[torch.as_tensor(rows, device="cuda")]), Cref, R, out_bf16=False)
     assert rep["ok"], rep
