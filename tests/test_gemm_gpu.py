@@ -643,3 +643,38 @@ def test_tensor_map_cache_hits_on_repeated_calls(pw):
     torch.cuda.synchronize()
     h1, m1 = pw.capi.gemm_bf16_tensor_map_cache_stats()
     assert (h1 - h0, m1 - m0) == (3, 0)
+
+
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_large_unaligned_c(pw, out):
+    """C that tensor stores cannot address (odd ldc; a base one element off a 16-byte boundary)
+    on a multi-wave GEMM: the result, with beta = 0 and beta = 1, matches the oracle and the
+    columns past N and the elements around C keep their canaries."""
+    _plan(pw, -1)
+    M, N, K = 2100, 2050, 320
+    A = matrix_bf16(1801, M, K)
+    B = matrix_bf16(1802, N, K)
+    ldc = 2053
+    c0bits = matrix_bf16(1803, M, N, ld=ldc)
+    c0 = torch.from_numpy(bf16_bits_to_f64(c0bits)).to(out)
+    for beta in (0.0, 1.0):
+        C, buf = _run(pw, A, B, M, N, K, out=out, alpha=0.5, beta=beta, c0=c0, ldc=ldc)
+        Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, c0=c0bits if beta else None, alpha=0.5, beta=beta)
+        rep = check(values_f64(C), Cref, R, out_bf16=out == torch.bfloat16)
+        assert rep["ok"], (beta, rep)
+        pad_before = c0[:, N:].to(torch.float32).numpy()
+        pad_after = buf[:, N:].cpu().to(torch.float32).numpy()
+        assert np.array_equal(np.isnan(pad_before), np.isnan(pad_after))
+        assert np.array_equal(pad_before[~np.isnan(pad_before)], pad_after[~np.isnan(pad_after)])
+    # aligned ldc, base one element past a 16-byte boundary
+    ldc = 2056
+    full = torch.full((M * ldc + 8,), float("nan"), dtype=out, device="cuda")
+    C = full[1:1 + M * ldc].view(M, ldc)[:, :N]
+    pw.gemm_bf16(to_dev_bf16(A), to_dev_bf16(B), C, alpha=0.5, beta=0.0)
+    torch.cuda.synchronize()
+    assert pw.device_status() == 0
+    Cref, R = oracle.gemm(A, B, M=M, N=N, K=K, alpha=0.5)
+    rep = check(values_f64(C), Cref, R, out_bf16=out == torch.bfloat16)
+    assert rep["ok"], rep
+    assert torch.isnan(full[0]).item() and torch.isnan(full[1 + M * ldc:]).all().item()
+    assert torch.isnan(full[1:1 + M * ldc].view(M, ldc)[:, N:]).all().item()
