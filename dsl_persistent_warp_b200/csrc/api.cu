@@ -1046,9 +1046,9 @@ gemm_status_t guarded(const Req& r, Workspace w) {
 }
 
 // Candidate configurations for a request: every plan that serves it (resident-A plans as they
-// are), unsplit and with each valid split of K through the workspace (2, 4, 8 slices) or across
-// a cluster (2, 4, 8 CTAs, one-CTA plans), and raster groups of 8, 16 and 32 m-blocks when the
-// tiles fill more than two waves.
+// are), unsplit, with stream-K where it applies, with each valid split of K through the workspace
+// (2, 4, 8 slices) or across a cluster (2, 4, 8 CTAs or 2, 4 CTA pairs), and raster groups of 8,
+// 16 and 32 m-blocks when the tiles fill more than two waves.
 std::vector<Choice> candidates(const Req& rg, int sms, const int* ccap, bool dedup) {
     std::vector<Choice> c;
     for (int i = 0; i < kNumPlans; ++i) {

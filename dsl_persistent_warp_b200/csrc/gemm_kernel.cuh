@@ -96,8 +96,8 @@ struct KParams {
     int splits;              // K slices per tile (split-K; <= 1: none).  Work unit u covers tile
                              // u / splits and k-blocks [s*kb_per_split, (s+1)*kb_per_split), s = u % splits
     int kb_per_split;        // k-blocks per slice (global or cluster split-K)
-    int csplit;              // cluster split-K (one-CTA plans): K slices per tile, computed by the
-                             // csplit CTAs of one thread-block cluster, one slice each; the partial
+    int csplit;              // cluster split-K: K slices per tile, computed by the csplit CTAs (CTA
+                             // pairs) of one thread-block cluster, one slice each; the partial
                              // sums are added through distributed shared memory (<= 1: none)
     int sk_tiles;            // stream-K: tiles [0, sk_tiles) are computed as K ranges spread evenly
                              // over sk_clusters clusters (0: none), the rest whole
