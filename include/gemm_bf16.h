@@ -190,8 +190,9 @@ GEMM_API gemm_status_t gemm_bf16_device_status(struct CUstream_st* stream);
  * 8; workspace) spreads the last wave's tiles over every cluster as equal ranges of k-blocks;
  * a tile cut by several ranges is added up like a workspace split.
  * All of them add the parts in a fixed order, so results stay bitwise reproducible.  The plan and
- * the split come from a cost model; environment variables read at every call override it for
- * sweeps and tests:
+ * the split come from the tuning table when gemm_autotune measured the problem, else from a cost
+ * model whose choice is kept per problem for later calls.  A forced plan or any of these
+ * environment variables (read at every call; for sweeps and tests) bypasses both:
  *   GEMM_BF16_SPLIT_K=s        (1..8) s workspace slices wherever the plan and K allow it
  *                              (1: no split of either kind unless the next variable forces one)
  *   GEMM_BF16_CLUSTER_SPLIT=s  (2, 4, 8) cluster split-K with s slices where the plan takes it;
