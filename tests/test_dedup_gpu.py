@@ -55,7 +55,7 @@ def test_dedup_matches_the_oracle(pw, case):
         assert rep["ok"], (out, beta, rep)
 
 
-@pytest.mark.parametrize("plan", [0, 2, 7])
+@pytest.mark.parametrize("plan", [0, 2, 7, 8])
 def test_dedup_bitwise_equals_the_expanded_batch(pw, plan):
     """The same tile plan on the expanded batch X[b] = X[index[b]] gives the same bits."""
     pw.capi.gemm_bf16_set_plan(plan)
