@@ -45,6 +45,12 @@
 #ifndef PW_EPI8_NSUB2
 #define PW_EPI8_NSUB2 1
 #endif
+// Resident-A plans (short mainloops, so the epilogue sets the pace) use 8 epilogue warps, two per
+// TMEM lane quarter, each storing half of the columns (1), or 4 (0).  B200, RecSys 2048 x
+// (256x512 . 512x128): 94.3 -> 85.6 us; 512 distinct entries x 4 items, dedup: 59.8 -> 54.3 us.
+#ifndef PW_EPI8_ARES
+#define PW_EPI8_ARES 1
+#endif
 
 namespace pw {
 
@@ -148,8 +154,9 @@ struct Tile {
     // store of one chunk overlaps the next chunk's TMEM load and conversion); for two sub-tiles
     // and 16-bit output, 8 warps (two per quarter, each half of the columns, one buffer each),
     // which drain the tile's accumulators into registers before storing so that the next tile's
-    // MMAs start sooner (B200, 8192^3: the MMAs' wait between tiles 7.3 -> 4.0 us, 2-3 % faster).
-    static constexpr int EPI_WARPS = (NSUB == 2 && OUT != OUT_F32 && PW_EPI8_NSUB2) ? 8 : 4;
+    // MMAs start sooner (B200, 8192^3: the MMAs' wait between tiles 7.3 -> 4.0 us, 2-3 % faster);
+    // for resident A, 8 warps storing chunk by chunk (twice the stores in flight).
+    static constexpr int EPI_WARPS = ((NSUB == 2 && OUT != OUT_F32 && PW_EPI8_NSUB2) || (ARES && PW_EPI8_ARES)) ? 8 : 4;
     static constexpr int EPI_HALVES = EPI_WARPS / 4;          // warps sharing a lane quarter
     static constexpr int STG_BUFS = 8 / EPI_WARPS;            // staging buffers per warp
     static constexpr int THREADS = 32 * (2 + EPI_WARPS);
