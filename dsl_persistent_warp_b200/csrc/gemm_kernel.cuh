@@ -51,6 +51,13 @@
 #ifndef PW_EPI8_ARES
 #define PW_EPI8_ARES 1
 #endif
+// The same for the other 2-CTA plans whose CTA holds at least two epilogue chunks per slot (1),
+// or 4 warps (0).  B200: 4099^3 (beta = 1, row-by-row epilogue) 174.4 -> 168.3 us, 2048^2 x 8192
+// 61.4 -> 60.4 us; on the one-CTA plans it was neutral or slower (1024^2 x 8192 cut over a
+// cluster of 4: 31.7 -> 32.8 us).
+#ifndef PW_EPI8_PAIR
+#define PW_EPI8_PAIR 1
+#endif
 
 namespace pw {
 
@@ -155,8 +162,11 @@ struct Tile {
     // and 16-bit output, 8 warps (two per quarter, each half of the columns, one buffer each),
     // which drain the tile's accumulators into registers before storing so that the next tile's
     // MMAs start sooner (B200, 8192^3: the MMAs' wait between tiles 7.3 -> 4.0 us, 2-3 % faster);
-    // for resident A, 8 warps storing chunk by chunk (twice the stores in flight).
-    static constexpr int EPI_WARPS = ((NSUB == 2 && OUT != OUT_F32 && PW_EPI8_NSUB2) || (ARES && PW_EPI8_ARES)) ? 8 : 4;
+    // for resident A and the other wide 2-CTA tiles, 8 warps storing chunk by chunk (twice the
+    // stores in flight).
+    static constexpr int EPI_WARPS = ((NSUB == 2 && OUT != OUT_F32 && PW_EPI8_NSUB2) || (ARES && PW_EPI8_ARES) ||
+                                      (CG == 2 && PW_EPI8_PAIR && BN / CG >= 2 * (OUT == OUT_F32 ? 32 : 64)))
+                                         ? 8 : 4;
     static constexpr int EPI_HALVES = EPI_WARPS / 4;          // warps sharing a lane quarter
     static constexpr int STG_BUFS = 8 / EPI_WARPS;            // staging buffers per warp
     static constexpr int THREADS = 32 * (2 + EPI_WARPS);
@@ -1059,7 +1069,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
         if constexpr (T::CSPLIT_OK) {
             if (CS > 1) {
                 // Cluster split-K reduction.  Once every CTA of the cluster has its partial tile in
-                // its shared memory, the 4*CS epilogue warps of the CTAs holding the same 128 rows
+                // its shared memory, the EPI_WARPS*CS epilogue warps of the CTAs holding the same 128 rows
                 // (one per slice) share those rows' (lane quarter, column chunk) items; each adds
                 // the CS partials of its item in slice order 0..CS-1, reading them through
                 // distributed shared memory, and runs the normal alpha/beta epilogue on the sum.
@@ -1070,7 +1080,7 @@ __global__ void __launch_bounds__(Tile<CG, BN, NSUB, STAGES, BK, B_MN, OUT, ARES
                     int b, mb, nb;
                     decode_tile(p, cluster_id, b, mb, nb);
                     constexpr int CH = BN / T::STG_COLS;  // column chunks of the tile
-                    for (int it = (int)crank * 4 + ew; it < 4 * CH; it += 4 * CS) {
+                    for (int it = (int)crank * T::EPI_WARPS + ew; it < 4 * CH; it += T::EPI_WARPS * CS) {
                         const int qq = it & 3, c = it >> 2;
                         const int row0 = mb * T::BM + (int)rank * 128 + 32 * qq;
                         float v[T::STG_COLS];
